@@ -1,0 +1,203 @@
+/*
+ * veda.h - C ABI of the Veda tile-skip sparse-attention path for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute is defined by the page "veda_core.py" (ComfyUI-FunPack node pack, "Veda
+ * sparse attention, the torch half"); each declaration below names the section and function it
+ * follows. One attention layer is, per group of heads that share a target tile box:
+ *
+ *     veda_plan      -> tile layout of the packed sequence + per-row budgets   (host, once per geometry)
+ *     veda_gather    -> Q, K (and V) in tile order; Q/K pooled to [mean|max|min] per tile
+ *     veda_score     -> per-head projected tile-pair scores
+ *     veda_select    -> kept key tiles of every video query tile (ascending index lists)
+ *     veda_attend    -> flash attention over the kept K/V tiles, written back to packed row order
+ *
+ * Conventions shared by every call
+ *  - Every pointer named "device" is CUDA device memory owned by the caller; the library never frees
+ *    it and keeps no reference to it after the call returns. Host pointers are read during the call only.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Device calls are
+ *    asynchronous: they enqueue kernels and return; errors detected inside a kernel (a bounded wait
+ *    that expired, a malformed kept list) are latched in a per-device error word that
+ *    veda_sync_status() reads.
+ *  - bf16 tensors are IEEE bfloat16 (2 bytes). Strided [S, H, D] tensors need a unit stride on D,
+ *    strides on S and H that are multiples of 8 elements, and a 16-byte aligned base.
+ *  - Tile-ordered tensors are head-major: [n_heads, N, D] with N = 128 * n_tiles rows per head, row
+ *    r of head h at ((h * N) + r) * D. Padding slots hold zeros.
+ *  - Return value: VEDA_OK or an error code; the text of the last error of the calling thread is
+ *    returned by veda_last_error(). There is no fallback path: a call that cannot run fails.
+ */
+#ifndef VEDA_H
+#define VEDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VEDA_TILE 128
+
+/* status codes */
+#define VEDA_OK 0
+#define VEDA_ERR_INVALID 1     /* a layout, budget, shape, stride or pointer the method cannot use */
+#define VEDA_ERR_CUDA 2        /* a CUDA runtime/driver call failed */
+#define VEDA_ERR_TIMEOUT 3     /* a bounded device-side wait expired (the kernel stopped cleanly) */
+#define VEDA_ERR_UNSUPPORTED 4 /* not an sm_100 device, or a size beyond a kernel's limit */
+#define VEDA_ERR_BAD_LIST 5    /* a kept list was out of range or not ascending (device check) */
+
+/* budget kinds: exactly one must be set (veda_core.py, "budgets": a budget is (ratio, tiles)) */
+#define VEDA_BUDGET_RATIO 1
+#define VEDA_BUDGET_TILES 2
+
+typedef struct veda_layout veda_layout; /* opaque; created by veda_plan, freed by veda_layout_destroy */
+
+/* A span of packed rows forming a row-major 3D grid (t, h, w), w fastest. A zero box (st = sh = sw = 0)
+ * asks for the least-padding box of the grid (veda_core.py, "tiles", least_padding_shape). */
+typedef struct {
+    int64_t start;
+    int32_t t, h, w;
+    int32_t st, sh, sw;
+} veda_span;
+
+/* kind = VEDA_BUDGET_RATIO: keep `ratio` of the key tiles (at equal kernel cost);
+ * kind = VEDA_BUDGET_TILES: keep exactly `tiles` key tiles per query tile. Any other kind is invalid
+ * (neither or both set). veda_core.py, "budgets": sparsity_budget, keeps_all, _per_row. */
+typedef struct {
+    int32_t kind;
+    double ratio;
+    int64_t tiles;
+} veda_budget;
+
+/* One key-column block with its own top-k (veda_core.py, "selection", column_blocks and _split). */
+typedef struct {
+    int32_t start, stop;  /* video key tiles [start, stop) */
+    int32_t keeps_all;    /* 1: every non-empty tile of the block is kept */
+    int32_t k_lo, k_hi;   /* per-row kept count is k_lo or k_lo + 1 (Bresenham) */
+    double frac;          /* fractional budget spread by the Bresenham pattern */
+    double row_budget;    /* the fractional per-row budget before the split */
+} veda_block_desc;
+
+typedef struct {
+    int64_t seq_len;      /* packed rows S */
+    int64_t n_slots;      /* N = 128 * n_tiles */
+    int32_t n_video;      /* span tiles (references first, then the target) */
+    int32_t n_ref;        /* reference tiles (0 when references are untiled) */
+    int32_t n_global;     /* tiles of the uncovered ("global") rows, after the span tiles */
+    int32_t n_tiles;      /* n_video + n_global */
+    int32_t n_kv_ok;      /* tiles holding at least one real row */
+    int32_t n_global_ok;  /* non-empty global tiles */
+    int32_t max_kept;     /* width of one kept-list row (an upper bound on any video row's count) */
+    int32_t tile_refs;    /* 1 when reference spans are tiled, 0 when their rows are global */
+    int64_t ref_tokens, target_tokens;
+    int32_t target_box[3];
+    int32_t n_blocks;     /* 1 (target) or 2 (references, target) */
+    veda_block_desc blocks[2];
+} veda_layout_desc;
+
+/* ------------------------------------------------------------------------------------------ host */
+
+/* Builds the tile layout of one head group (veda_core.py, "tiles", build_layout and span_tiles;
+ * "one layer", attention: references are tiled at their least-padding box unless the reference
+ * budget keeps all, in which case their rows become global rows).
+ *  spans   host [n_spans]: references in packed order, then the target span (last). The target's box is
+ *          the head group's box; a reference box of zero means least-padding (any other is honoured).
+ *  seq_len packed rows S; every row no (tiled) span covers is a global row.
+ *  generated / reference: budgets of the target block and of the reference block.
+ *  out     receives the new layout. Device copies of its index data are made on first device use,
+ *          once per device.
+ * Errors: VEDA_ERR_INVALID for no spans, spans out of packed order or overlapping or running past
+ * seq_len, a box that is not a power-of-two (t,h,w) with t*h*w = 128, and a budget with neither or
+ * both kinds set, a negative ratio or a tile count below 0. */
+int veda_plan(const veda_span* spans, int32_t n_spans, int64_t seq_len, veda_budget generated,
+              veda_budget reference, veda_layout** out);
+
+/* Sizes and budget split of a layout (host). */
+int veda_layout_info(const veda_layout* layout, veda_layout_desc* out);
+
+/* Copies the layout's index data to host arrays; any pointer may be NULL.
+ *  perm         [n_slots] int32: packed row of each tile slot, -1 on padding (veda_core.py, build_layout)
+ *  valid_count  [n_tiles] int32: real rows per tile (a prefix of the tile)
+ *  allowed      [n_blocks * n_video] int32: per block, the kept count k_lo + extra(row) of every video
+ *               query row (veda_core.py, "selection", select with _bresenham); n_block_cols for a
+ *               keeps-all block. */
+int veda_layout_export(const veda_layout* layout, int32_t* perm, int32_t* valid_count, int32_t* allowed);
+
+/* Frees a layout and its device copies (on every device that used it). NULL is ignored. */
+void veda_layout_destroy(veda_layout* layout);
+
+/* The least-padding box of a grid (veda_core.py, "tiles", least_padding_shape): among the power-of-two
+ * boxes that fit the grid (all 36 if none fits), fewest tiles, then most cubic, then lexicographic. */
+int veda_least_padding_box(int32_t t, int32_t h, int32_t w, int32_t box_out[3]);
+
+/* ---------------------------------------------------------------------------------------- device */
+
+/* Tile-order gather with the pooled features fused in (veda_core.py, "tiles", gather; "predictor", pool).
+ *  x          device bf16 [S, H_total, D] with element strides x_strides[3] (S, H, D).
+ *  heads      device int32 [n_heads]: which of the H_total heads form this group (any order).
+ *  x_t        device bf16 [n_heads, N, D] out: x_t[h, i] = x[perm[i], heads[h]], zero on padding.
+ *  feats      device fp32 [n_heads, n_video, 3D] out, or NULL to skip pooling: per video tile and head
+ *             [mean | max | min] over the tile's real rows (0 for an empty tile); mean = fp32 sum / count.
+ * D must be 64 or 128. */
+int veda_gather(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, void* stream);
+
+/* Workspace bytes veda_score needs (projected features of Q and K): 2 * n_heads * n_video * D * 4. */
+size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim);
+
+/* Tile-pair logits (veda_core.py, "predictor", logits): per head, q_hat = fq @ Pq + fq[:, :D],
+ * k_hat = fk @ Pk + fk[:, :D], scores = q_hat @ k_hat^T / sqrt(D), all fp32.
+ *  feats_q/k  device fp32 [n_heads, n_video, 3D] (from veda_gather).
+ *  proj_q/k   device fp32 [n_heads, 3D, D]: the group's heads' projections, in the group's head order.
+ *  workspace  device, at least veda_score_workspace_bytes(), 16-byte aligned.
+ *  scores     device fp32 [n_heads, n_video, n_video] out. */
+int veda_score(const veda_layout* layout, const float* feats_q, const float* feats_k, int32_t n_heads,
+               int32_t dim, const float* proj_q, const float* proj_k, void* workspace,
+               size_t workspace_bytes, float* scores, void* stream);
+
+/* Head-aware top-k (veda_core.py, "selection", select, block_mask and tile_index_list).
+ * Per head and video query row, per column block: empty key tiles are never kept; the row's own tile
+ * is kept first when it lies in the block; the other columns are ranked by (score descending, column
+ * ascending) and the first k_lo + extra(row) are kept (all non-empty columns for a keeps-all block).
+ * A NaN or -inf score is never kept. Every non-empty global tile is appended.
+ *  scores     device fp32 [n_heads, n_video, n_video] (any source).
+ *  kept_idx   device int32 [n_heads, n_video, max_kept] out: ascending tile ids; entries past the count
+ *             are left untouched.
+ *  kept_cnt   device int32 [n_heads, n_video] out.
+ * Global query rows are dense over every non-empty tile and need no list.
+ * Limit: a column block of at most 16384 tiles (VEDA_ERR_UNSUPPORTED beyond). */
+int veda_select(const veda_layout* layout, const float* scores, int32_t n_heads, int32_t* kept_idx,
+                int32_t* kept_cnt, void* stream);
+
+/* Block-sparse flash attention over the kept tiles, scattered back to packed rows (veda_core.py,
+ * "selection", reference_attend: scale D^-0.5, key slots restricted to real rows, a row that sees no
+ * key gives 0; "tiles", scatter_).
+ *  q_t, k_t, v_t  device bf16 [n_heads, N, D] tile order (from veda_gather).
+ *  kept_idx/cnt   as written by veda_select (or any lists in that format: ids ascending in
+ *                 [0, n_tiles), count <= max_kept; a malformed row is cut at its first bad entry and
+ *                 latched as VEDA_ERR_BAD_LIST).
+ *  out            device bf16 [S, H_total, D] with element strides out_strides[3]: rows of this group's
+ *                 heads (heads[h]) are overwritten; padding slots are dropped.
+ * D must be 64 or 128. Runs bf16 tensor-core MMAs (tcgen05) with fp32 accumulation and an fp32 online
+ * softmax; needs an sm_100 device. */
+int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
+                int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt,
+                void* out, const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
+                void* stream);
+
+/* Synchronizes `stream`, then reads and clears this device's latched kernel error word.
+ * Returns VEDA_OK, VEDA_ERR_TIMEOUT, VEDA_ERR_BAD_LIST or VEDA_ERR_CUDA. */
+int veda_sync_status(void* stream);
+
+/* Text of the calling thread's last error ("" if none). Valid until the thread's next veda_* call. */
+const char* veda_last_error(void);
+
+/* VEDA_OK when the current device is sm_100 (B200 class), else VEDA_ERR_UNSUPPORTED / VEDA_ERR_CUDA. */
+int veda_device_check(void);
+
+/* Upper bound, in nanoseconds, of every bounded device-side wait (default 1e9). Process-wide. */
+void veda_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VEDA_H */

@@ -1,0 +1,210 @@
+"""ctypes binding of libveda (include/veda.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls. Device tensors are torch CUDA tensors;
+their data pointers and strides are passed as plain integers. Nothing is computed in Python: when the
+library is missing or the device is not an sm_100 part, calls raise instead of falling back.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+VEDA_OK, VEDA_ERR_INVALID, VEDA_ERR_CUDA, VEDA_ERR_TIMEOUT, VEDA_ERR_UNSUPPORTED, VEDA_ERR_BAD_LIST = range(6)
+VEDA_BUDGET_RATIO, VEDA_BUDGET_TILES = 1, 2
+TILE = 128
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libveda.so")
+
+EXPORTS = [
+    "veda_plan", "veda_layout_info", "veda_layout_export", "veda_layout_destroy", "veda_least_padding_box",
+    "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_select", "veda_attend",
+    "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
+]
+
+
+class VedaError(RuntimeError):
+    """A libveda call failed; ``code`` is the VEDA_ERR_* status."""
+
+    def __init__(self, code, msg):
+        super().__init__(f"[veda {code}] {msg}")
+        self.code = code
+
+
+class Span(C.Structure):
+    _fields_ = [("start", C.c_int64), ("t", C.c_int32), ("h", C.c_int32), ("w", C.c_int32),
+                ("st", C.c_int32), ("sh", C.c_int32), ("sw", C.c_int32)]
+
+
+class Budget(C.Structure):
+    _fields_ = [("kind", C.c_int32), ("ratio", C.c_double), ("tiles", C.c_int64)]
+
+
+class BlockDesc(C.Structure):
+    _fields_ = [("start", C.c_int32), ("stop", C.c_int32), ("keeps_all", C.c_int32), ("k_lo", C.c_int32),
+                ("k_hi", C.c_int32), ("frac", C.c_double), ("row_budget", C.c_double)]
+
+
+class LayoutDesc(C.Structure):
+    _fields_ = [("seq_len", C.c_int64), ("n_slots", C.c_int64), ("n_video", C.c_int32), ("n_ref", C.c_int32),
+                ("n_global", C.c_int32), ("n_tiles", C.c_int32), ("n_kv_ok", C.c_int32),
+                ("n_global_ok", C.c_int32), ("max_kept", C.c_int32), ("tile_refs", C.c_int32),
+                ("ref_tokens", C.c_int64), ("target_tokens", C.c_int64), ("target_box", C.c_int32 * 3),
+                ("n_blocks", C.c_int32), ("blocks", BlockDesc * 2)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise VedaError(VEDA_ERR_UNSUPPORTED, f"libveda.so is not built ({LIB_PATH}); run "
+                            "`python -m learned_block_sparse_tile_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        p, i32, i64, vp = C.c_void_p, C.c_int32, C.c_int64, C.c_void_p
+        L.veda_plan.argtypes = [C.POINTER(Span), i32, i64, Budget, Budget, C.POINTER(vp)]
+        L.veda_layout_info.argtypes = [vp, C.POINTER(LayoutDesc)]
+        L.veda_layout_export.argtypes = [vp, p, p, p]
+        L.veda_layout_destroy.argtypes = [vp]
+        L.veda_layout_destroy.restype = None
+        L.veda_least_padding_box.argtypes = [i32, i32, i32, C.POINTER(C.c_int32)]
+        L.veda_gather.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, vp]
+        L.veda_score_workspace_bytes.argtypes = [vp, i32, i32]
+        L.veda_score_workspace_bytes.restype = C.c_size_t
+        L.veda_score.argtypes = [vp, p, p, i32, i32, p, p, p, C.c_size_t, p, vp]
+        L.veda_select.argtypes = [vp, p, i32, p, p, vp]
+        L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
+        L.veda_sync_status.argtypes = [vp]
+        L.veda_last_error.restype = C.c_char_p
+        L.veda_set_wait_timeout_ns.argtypes = [C.c_uint64]
+        L.veda_set_wait_timeout_ns.restype = None
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != VEDA_OK:
+        raise VedaError(rc, lib().veda_last_error().decode(errors="replace"))
+
+
+def _budget(b):
+    """(ratio, tiles) pair -> Budget. Exactly one must be set; the library rejects the rest."""
+    ratio, tiles = b
+    kind = (VEDA_BUDGET_RATIO if ratio is not None else 0) | (VEDA_BUDGET_TILES if tiles is not None else 0)
+    return Budget(kind, float(ratio) if ratio is not None else 0.0, int(tiles) if tiles is not None else 0)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return C.c_void_p(getattr(stream, "cuda_stream", stream))
+
+
+def _ptr(t):
+    return C.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _strides(t):
+    return (C.c_int64 * 3)(*t.stride())
+
+
+class Layout:
+    """Owns a ``veda_layout*`` (freed on garbage collection)."""
+
+    def __init__(self, handle):
+        self.handle = C.c_void_p(handle)
+        d = LayoutDesc()
+        _check(lib().veda_layout_info(self.handle, C.byref(d)))
+        self.desc = d
+        self.n_video, self.n_ref, self.n_global = d.n_video, d.n_ref, d.n_global
+        self.n_tiles, self.n_slots, self.max_kept = d.n_tiles, d.n_slots, d.max_kept
+        self.n_kv_ok, self.n_global_ok, self.seq_len = d.n_kv_ok, d.n_global_ok, d.seq_len
+        self.blocks = [(d.blocks[b].start, d.blocks[b].stop, bool(d.blocks[b].keeps_all), d.blocks[b].k_lo,
+                        d.blocks[b].k_hi, d.blocks[b].frac, d.blocks[b].row_budget) for b in range(d.n_blocks)]
+
+    def __del__(self):
+        if getattr(self, "handle", None) and self.handle.value and _lib is not None:
+            _lib.veda_layout_destroy(self.handle)
+            self.handle = None
+
+
+def veda_plan(spans, seq_len, generated, reference):
+    """``spans``: [(start, (t, h, w), box or None)] references in packed order, target last."""
+    arr = (Span * len(spans))()
+    for i, (start, grid, box) in enumerate(spans):
+        b = (0, 0, 0) if box is None else box
+        arr[i] = Span(int(start), *[int(g) for g in grid], *[int(x) for x in b])
+    out = C.c_void_p()
+    _check(lib().veda_plan(arr, len(spans), int(seq_len), _budget(generated), _budget(reference), C.byref(out)))
+    return Layout(out.value)
+
+
+def veda_layout_info(layout):
+    return layout.desc
+
+
+def veda_layout_export(layout):
+    """(perm [N], valid_count [n_tiles], allowed [n_blocks, n_video]) as int32 numpy arrays."""
+    d = layout.desc
+    perm = np.empty(d.n_slots, np.int32)
+    vc = np.empty(d.n_tiles, np.int32)
+    allowed = np.empty((d.n_blocks, d.n_video), np.int32)
+    _check(lib().veda_layout_export(layout.handle, perm.ctypes.data, vc.ctypes.data, allowed.ctypes.data))
+    return perm, vc, allowed
+
+
+def veda_least_padding_box(grid):
+    out = (C.c_int32 * 3)()
+    _check(lib().veda_least_padding_box(int(grid[0]), int(grid[1]), int(grid[2]), out))
+    return tuple(out)
+
+
+def veda_gather(layout, x, heads, x_t, feats=None, stream=None):
+    """x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; x_t: bf16 [n, N, D]; feats: fp32 [n, n_video, 3D] or None."""
+    _check(lib().veda_gather(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
+                             heads.numel(), _ptr(x_t), _ptr(feats), _stream(stream)))
+
+
+def veda_score_workspace_bytes(layout, n_heads, dim):
+    return int(lib().veda_score_workspace_bytes(layout.handle, n_heads, dim))
+
+
+def veda_score(layout, feats_q, feats_k, proj_q, proj_k, workspace, scores, stream=None):
+    n_heads, dim = proj_q.shape[0], proj_q.shape[2]
+    _check(lib().veda_score(layout.handle, _ptr(feats_q), _ptr(feats_k), n_heads, dim, _ptr(proj_q), _ptr(proj_k),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(scores),
+                            _stream(stream)))
+
+
+def veda_select(layout, scores, kept_idx, kept_cnt, stream=None):
+    _check(lib().veda_select(layout.handle, _ptr(scores), scores.shape[0], _ptr(kept_idx), _ptr(kept_cnt),
+                             _stream(stream)))
+
+
+def veda_attend(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, stream=None):
+    """q_t/k_t/v_t: bf16 [n, N, D]; out: bf16 [S, H, D] (strided ok); heads: int32 [n] cuda."""
+    _check(lib().veda_attend(layout.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), q_t.shape[0], q_t.shape[2],
+                             _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1], _ptr(heads),
+                             _stream(stream)))
+
+
+def veda_sync_status(stream=None):
+    """Synchronizes the stream and returns the latched kernel status code (does not raise)."""
+    return int(lib().veda_sync_status(_stream(stream)))
+
+
+def veda_last_error():
+    return lib().veda_last_error().decode(errors="replace")
+
+
+def veda_device_check():
+    _check(lib().veda_device_check())
+
+
+def veda_set_wait_timeout_ns(ns):
+    lib().veda_set_wait_timeout_ns(int(ns))

@@ -1,0 +1,126 @@
+// Tile-order gather of one [S, H, D] bf16 tensor with the per-tile [mean | max | min] pooling fused in.
+// veda_core.py (ComfyUI-FunPack): "tiles", gather (x[perm, heads], zero on padding slots) and
+// "predictor", pool (mean = fp32 sum of the tile's real rows / their count; max and min over the real
+// rows only; zero for a tile with no real row).
+//
+// One CTA per (tile, head): 256 threads move the tile's 128 rows of D bf16 with 16-byte loads (each
+// row is one contiguous 2*D-byte run of the source), keep them in registers, write them to the
+// head-major tile-ordered output and reduce them column-wise in the same pass. HBM bound.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+namespace veda {
+
+struct GatherArgs {
+    const __nv_bfloat16* x;
+    int64_t s0, s1;               // element strides of x on S and H (D stride is 1)
+    const int32_t* heads;         // [n_heads]
+    const int32_t* perm;          // [n_slots]
+    const int32_t* valid_count;   // [n_tiles]
+    __nv_bfloat16* x_t;           // [n_heads, n_slots, D]
+    float* feats;                 // [n_heads, n_video, 3D] or null
+    int64_t n_slots;
+    int32_t n_video;
+    int32_t h_total;
+    int* err;                     // latched error bits; bit 4 = head index out of range
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
+    constexpr int kTpr = D / 8;          // threads per row (8 bf16 = 16 bytes each)
+    constexpr int kRpp = 256 / kTpr;     // rows per pass
+    constexpr int kPasses = 128 / kRpp;  // passes over the tile
+    constexpr int kWarps = 8;
+    __shared__ float red[3][kWarps][D];
+
+    const int tile = blockIdx.x, hh = blockIdx.y;
+    const int tid = threadIdx.x, c = tid % kTpr, r0 = tid / kTpr;
+    const int64_t head = __ldg(a.heads + hh);
+    if (head < 0 || head >= a.h_total) {  // uniform across the CTA
+        if (threadIdx.x == 0) atomicOr(a.err, 4);
+        return;
+    }
+    const int vc = __ldg(a.valid_count + tile);
+    const __nv_bfloat16* src = a.x + head * a.s1 + c * 8;
+
+    uint4 v[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        const int r = r0 + p * kRpp;
+        const int pr = __ldg(a.perm + int64_t(tile) * 128 + r);
+        v[p] = pr >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + int64_t(pr) * a.s0)) : make_uint4(0, 0, 0, 0);
+    }
+    __nv_bfloat16* dst = a.x_t + (int64_t(hh) * a.n_slots + int64_t(tile) * 128) * D + c * 8;
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) *reinterpret_cast<uint4*>(dst + int64_t(r0 + p * kRpp) * D) = v[p];
+
+    if (a.feats == nullptr || tile >= a.n_video) return;
+
+    float sum[8], mx[8], mn[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        sum[e] = 0.f;
+        mx[e] = -INFINITY;
+        mn[e] = INFINITY;
+    }
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        if (r0 + p * kRpp < vc) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                sum[2 * e] += f.x;
+                sum[2 * e + 1] += f.y;
+                mx[2 * e] = fmaxf(mx[2 * e], f.x);
+                mx[2 * e + 1] = fmaxf(mx[2 * e + 1], f.y);
+                mn[2 * e] = fminf(mn[2 * e], f.x);
+                mn[2 * e + 1] = fminf(mn[2 * e + 1], f.y);
+            }
+        }
+    }
+    // lanes that hold the same columns differ in the bits above log2(kTpr)
+#pragma unroll
+    for (int off = kTpr; off < 32; off <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            sum[e] += __shfl_xor_sync(0xffffffffu, sum[e], off);
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
+            mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], off));
+        }
+    }
+    const int warp = tid >> 5, lane = tid & 31;
+    if (lane < kTpr) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            red[0][warp][c * 8 + e] = sum[e];
+            red[1][warp][c * 8 + e] = mx[e];
+            red[2][warp][c * 8 + e] = mn[e];
+        }
+    }
+    __syncthreads();
+    if (tid < D) {
+        float s = 0.f, hi = -INFINITY, lo = INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            s += red[0][w][tid];
+            hi = fmaxf(hi, red[1][w][tid]);
+            lo = fminf(lo, red[2][w][tid]);
+        }
+        float* f = a.feats + (int64_t(hh) * a.n_video + tile) * (3 * D);
+        if (vc > 0) {
+            f[tid] = s / float(vc);
+            f[D + tid] = hi;
+            f[2 * D + tid] = lo;
+        } else {
+            f[tid] = 0.f;
+            f[D + tid] = 0.f;
+            f[2 * D + tid] = 0.f;
+        }
+    }
+}
+
+}  // namespace veda

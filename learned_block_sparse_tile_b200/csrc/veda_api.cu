@@ -1,0 +1,385 @@
+// C ABI entry points of libveda: argument checks, device copies of layouts, tensor maps and launches.
+// The kernels themselves live in gather.cuh, score.cuh, select.cuh and attend.cuh (one translation
+// unit, so they share the latched device error word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "veda_internal.h"
+#include "gather.cuh"
+#include "score.cuh"
+#include "select.cuh"
+#include "attend.cuh"
+
+namespace veda {
+
+constexpr int kErrBadHead = 4;
+
+__device__ int g_err;  // latched kernel error bits (kErrTimeout | kErrBadList | kErrBadHead)
+
+namespace {
+
+thread_local std::string t_error;
+std::atomic<uint64_t> g_timeout_ns{1000000000ull};
+
+struct DeviceState {
+    bool init = false;
+    int sms = 0;
+    int* err = nullptr;  // device address of g_err
+    bool attend_attr[2] = {false, false};
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(VEDA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+int device_state(DeviceState** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal beyond the library's table");
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    DeviceState& s = g_dev[dev];
+    if (!s.init) {
+        cudaDeviceProp p;
+        e = cudaGetDeviceProperties(&p, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+        if (p.major != 10 || p.minor != 0)
+            return fail(VEDA_ERR_UNSUPPORTED, "libveda needs an sm_100 (B200-class) device; found sm_" +
+                                                  std::to_string(p.major) + std::to_string(p.minor));
+        s.sms = p.multiProcessorCount;
+        e = cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), g_err);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+        s.init = true;
+    }
+    *out = &s;
+    return VEDA_OK;
+}
+
+// Device copy of a layout's index data on the current device (made on first use).
+int device_copy(const veda_layout* lay, const DeviceCopy** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal beyond the library's table");
+    std::lock_guard<std::mutex> g(lay->mu);
+    DeviceCopy& dc = lay->dev[dev];
+    if (!dc.ready) {
+        auto up = [&](int32_t** dst, const std::vector<int32_t>& src) -> cudaError_t {
+            const size_t bytes = std::max<size_t>(src.size(), 1) * sizeof(int32_t);
+            cudaError_t r = cudaMalloc(reinterpret_cast<void**>(dst), bytes);
+            if (r != cudaSuccess) return r;
+            if (!src.empty()) r = cudaMemcpy(*dst, src.data(), src.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+            return r;
+        };
+        if ((e = up(&dc.perm, lay->perm)) != cudaSuccess || (e = up(&dc.valid_count, lay->valid_count)) != cudaSuccess ||
+            (e = up(&dc.ok_list, lay->ok_list)) != cudaSuccess || (e = up(&dc.allowed, lay->allowed)) != cudaSuccess)
+            return cuda_fail(e, "uploading the layout");
+        dc.ready = true;
+    }
+    *out = &dc;
+    return VEDA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_strided(const int64_t* st, const void* base, const char* name) {
+    if (!st) return fail(VEDA_ERR_INVALID, std::string(name) + ": strides are NULL");
+    if (st[2] != 1 || st[0] % 8 != 0 || st[1] % 8 != 0 || st[0] <= 0 || st[1] <= 0 || !aligned16(base))
+        return fail(VEDA_ERR_INVALID, std::string(name) +
+                                          ": needs D stride 1, S and H strides positive multiples of 8, 16-byte base");
+    return VEDA_OK;
+}
+
+int launch_check(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return VEDA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D map over a head-major tile-ordered bf16 tensor viewed as [rows, D]: boxes of 128 rows x 64 columns
+// (128 bytes) with the 128-byte swizzle the MMA descriptors expect.
+int make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int dim) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[2] = {cuuint64_t(dim), cuuint64_t(rows)};
+    cuuint64_t gstride[1] = {cuuint64_t(dim) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+    return VEDA_OK;
+}
+
+}  // namespace
+
+int fail(int code, const std::string& msg) {
+    t_error = msg;
+    return code;
+}
+
+void clear_error() { t_error.clear(); }
+
+}  // namespace veda
+
+using namespace veda;
+
+extern "C" const char* veda_last_error(void) { return t_error.c_str(); }
+
+extern "C" void veda_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : 1; }
+
+extern "C" int veda_device_check(void) {
+    clear_error();
+    DeviceState* s;
+    return device_state(&s);
+}
+
+extern "C" void veda_layout_destroy(veda_layout* layout) {
+    if (!layout) return;
+    int cur = -1;
+    const bool have = cudaGetDevice(&cur) == cudaSuccess;
+    for (int d = 0; d < kMaxDevices; ++d) {
+        DeviceCopy& dc = layout->dev[d];
+        if (!dc.ready) continue;
+        if (cudaSetDevice(d) == cudaSuccess) {
+            cudaFree(dc.perm);
+            cudaFree(dc.valid_count);
+            cudaFree(dc.ok_list);
+            cudaFree(dc.allowed);
+        }
+    }
+    if (have) cudaSetDevice(cur);
+    delete layout;
+}
+
+extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                           int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, void* stream) {
+    clear_error();
+    if (!layout || !x || !heads || !x_t) return fail(VEDA_ERR_INVALID, "veda_gather: NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_gather: head_dim must be 64 or 128");
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_gather: head counts must be positive");
+    if (int rc = check_strided(x_strides, x, "veda_gather x")) return rc;
+    if (!aligned16(x_t) || (feats && !aligned16(feats))) return fail(VEDA_ERR_INVALID, "veda_gather: outputs need 16-byte alignment");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    const veda_layout_desc& d = layout->desc;
+    GatherArgs a;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.s0 = x_strides[0];
+    a.s1 = x_strides[1];
+    a.heads = heads;
+    a.perm = dc->perm;
+    a.valid_count = dc->valid_count;
+    a.x_t = static_cast<__nv_bfloat16*>(x_t);
+    a.feats = feats;
+    a.n_slots = d.n_slots;
+    a.n_video = d.n_video;
+    a.h_total = h_total;
+    a.err = ds->err;
+    dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dim == 128)
+        gather_pool_kernel<128><<<grid, 256, 0, s>>>(a);
+    else
+        gather_pool_kernel<64><<<grid, 256, 0, s>>>(a);
+    return launch_check("gather_pool_kernel");
+}
+
+extern "C" size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim) {
+    if (!layout || n_heads <= 0 || dim <= 0) return 0;
+    return size_t(2) * size_t(n_heads) * size_t(layout->desc.n_video) * size_t(dim) * sizeof(float);
+}
+
+extern "C" int veda_score(const veda_layout* layout, const float* feats_q, const float* feats_k, int32_t n_heads,
+                          int32_t dim, const float* proj_q, const float* proj_k, void* workspace,
+                          size_t workspace_bytes, float* scores, void* stream) {
+    clear_error();
+    if (!layout || !feats_q || !feats_k || !proj_q || !proj_k || !workspace || !scores)
+        return fail(VEDA_ERR_INVALID, "veda_score: NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_score: head_dim must be 64 or 128");
+    if (n_heads <= 0) return fail(VEDA_ERR_INVALID, "veda_score: n_heads must be positive");
+    if (workspace_bytes < veda_score_workspace_bytes(layout, n_heads, dim))
+        return fail(VEDA_ERR_INVALID, "veda_score: workspace smaller than veda_score_workspace_bytes()");
+    if (!aligned16(feats_q) || !aligned16(feats_k) || !aligned16(proj_q) || !aligned16(proj_k) ||
+        !aligned16(workspace) || !aligned16(scores))
+        return fail(VEDA_ERR_INVALID, "veda_score: buffers need 16-byte alignment");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const int nv = layout->desc.n_video;
+    float* qh = static_cast<float*>(workspace);
+    float* kh = qh + int64_t(n_heads) * nv * dim;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int side = 0; side < 2; ++side) {
+        GemmArgs g;
+        g.A = side ? feats_k : feats_q;
+        g.B = side ? proj_k : proj_q;
+        g.C = side ? kh : qh;
+        g.M = nv;
+        g.N = dim;
+        g.K = 3 * dim;
+        g.sA = int64_t(nv) * 3 * dim;
+        g.sB = int64_t(3) * dim * dim;
+        g.sC = int64_t(nv) * dim;
+        g.div = 1.f;
+        gemm_f32_kernel<false><<<dim3(unsigned((dim + 63) / 64), unsigned((nv + 63) / 64), unsigned(n_heads)), 256, 0, s>>>(g);
+    }
+    GemmArgs g;
+    g.A = qh;
+    g.B = kh;
+    g.C = scores;
+    g.M = nv;
+    g.N = nv;
+    g.K = dim;
+    g.sA = int64_t(nv) * dim;
+    g.sB = int64_t(nv) * dim;
+    g.sC = int64_t(nv) * nv;
+    g.div = float(std::sqrt(double(dim)));
+    gemm_f32_kernel<true><<<dim3(unsigned((nv + 63) / 64), unsigned((nv + 63) / 64), unsigned(n_heads)), 256, 0, s>>>(g);
+    return launch_check("gemm_f32_kernel");
+}
+
+extern "C" int veda_select(const veda_layout* layout, const float* scores, int32_t n_heads, int32_t* kept_idx,
+                           int32_t* kept_cnt, void* stream) {
+    clear_error();
+    if (!layout || !scores || !kept_idx || !kept_cnt) return fail(VEDA_ERR_INVALID, "veda_select: NULL argument");
+    if (n_heads <= 0) return fail(VEDA_ERR_INVALID, "veda_select: n_heads must be positive");
+    const veda_layout_desc& d = layout->desc;
+    int widest = 1;
+    for (int b = 0; b < d.n_blocks; ++b) widest = std::max(widest, d.blocks[b].stop - d.blocks[b].start);
+    if (widest > kSelectMaxCols)
+        return fail(VEDA_ERR_UNSUPPORTED, "veda_select: a column block wider than 16384 tiles");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    SelectArgs a;
+    a.scores = scores;
+    a.valid_count = dc->valid_count;
+    a.allowed = dc->allowed;
+    a.ok_list = dc->ok_list;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.n_video = d.n_video;
+    a.n_blocks = d.n_blocks;
+    a.max_kept = d.max_kept;
+    a.n_kv_ok = d.n_kv_ok;
+    a.n_global_ok = d.n_global_ok;
+    for (int b = 0; b < 2; ++b) {
+        a.blk_start[b] = b < d.n_blocks ? d.blocks[b].start : 0;
+        a.blk_stop[b] = b < d.n_blocks ? d.blocks[b].stop : 0;
+        a.blk_all[b] = b < d.n_blocks ? d.blocks[b].keeps_all : 0;
+    }
+    const size_t smem = size_t(widest) * sizeof(uint32_t);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(select_kernel)");
+    }
+    select_kernel<<<dim3(unsigned(d.n_video), unsigned(n_heads)), kSelectThreads, smem, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_check("select_kernel");
+}
+
+template <int D>
+static int launch_attend(DeviceState* ds, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const AttendArgs& a, cudaStream_t s) {
+    using C = AttendCfg<D>;
+    if (!ds->attend_attr[D == 128]) {
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
+        ds->attend_attr[D == 128] = true;
+    }
+    const int grid = std::max(1, std::min(a.n_items, ds->sms));
+    attend_kernel<D><<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, a);
+    return launch_check("attend_kernel");
+}
+
+extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
+                           int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                           const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
+    clear_error();
+    if (!layout || !q_t || !k_t || !v_t || !kept_idx || !kept_cnt || !out || !heads)
+        return fail(VEDA_ERR_INVALID, "veda_attend: NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_attend: head_dim must be 64 or 128");
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_attend: head counts must be positive");
+    if (int rc = check_strided(out_strides, out, "veda_attend out")) return rc;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t))
+        return fail(VEDA_ERR_INVALID, "veda_attend: tile-ordered inputs need 16-byte alignment");
+    const veda_layout_desc& d = layout->desc;
+    if (int64_t(n_heads) * d.n_slots >= (int64_t(1) << 31))
+        return fail(VEDA_ERR_UNSUPPORTED, "veda_attend: n_heads * N must stay below 2^31 rows");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    CUtensorMap mq, mk, mv;
+    const int64_t rows = int64_t(n_heads) * d.n_slots;
+    if (int rc = make_tile_map(&mq, q_t, rows, dim)) return rc;
+    if (int rc = make_tile_map(&mk, k_t, rows, dim)) return rc;
+    if (int rc = make_tile_map(&mv, v_t, rows, dim)) return rc;
+    AttendArgs a;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.ok_list = dc->ok_list;
+    a.valid_count = dc->valid_count;
+    a.perm = dc->perm;
+    a.heads = heads;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.out_s0 = out_strides[0];
+    a.out_s1 = out_strides[1];
+    a.n_slots = d.n_slots;
+    a.max_kept = d.max_kept;
+    a.n_ok = d.n_kv_ok;
+    a.n_tiles = d.n_tiles;
+    a.n_video = d.n_video;
+    a.n_global = d.n_global;
+    a.n_heads = n_heads;
+    a.h_total = h_total;
+    a.n_items = n_heads * d.n_tiles;
+    a.scale_log2 = float((1.0 / std::sqrt(double(dim))) * 1.4426950408889634);
+    a.timeout_ns = g_timeout_ns.load();
+    a.err = ds->err;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dim == 128 ? launch_attend<128>(ds, mq, mk, mv, a, s) : launch_attend<64>(ds, mq, mk, mv, a, s);
+}
+
+extern "C" int veda_sync_status(void* stream) {
+    clear_error();
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int bits = 0;
+    e = cudaMemcpyFromSymbol(&bits, g_err, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (bits) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_err, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    }
+    if (bits & kErrTimeout) return fail(VEDA_ERR_TIMEOUT, "a bounded device wait expired; the kernel stopped early");
+    if (bits & kErrBadList) return fail(VEDA_ERR_BAD_LIST, "a kept list was out of range or not ascending");
+    if (bits & kErrBadHead) return fail(VEDA_ERR_INVALID, "a head index was outside [0, H_total)");
+    return VEDA_OK;
+}

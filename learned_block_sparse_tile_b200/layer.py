@@ -1,0 +1,96 @@
+"""One Veda attention layer on the C ABI (veda_core.py, "one layer", attention).
+
+For each group of heads sharing a target tile box: plan (cached), gather Q and K to tile order with
+pooling, score, select, gather V, attend with the scatter fused. PyTorch only allocates device buffers
+and supplies the stream; every step runs in libveda's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+class VedaLayer:
+    """Plans and buffers for one layer geometry.
+
+    seq_len      packed rows S
+    ref_spans    [(start, (t, h, w))] reference spans in packed order (tiled at their least-padding box
+                 unless the reference budget keeps all)
+    target       (start, (t, h, w)) the generated span (last)
+    head_shapes  per head: a (t, h, w) box or None for the target's least-padding box
+    budgets      (generated, reference), each a (ratio, tiles) pair with exactly one set
+    """
+
+    LAUNCHES_PER_GROUP = 8  # gather q, gather k, 3 score GEMMs, select, gather v, attend
+
+    def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda"):
+        self.seq_len, self.heads, self.dim = int(seq_len), int(heads), int(dim)
+        self.device = torch.device(device)
+        lps = L.veda_least_padding_box(target[1])
+        groups = {}
+        for h, s in enumerate(head_shapes):
+            groups.setdefault(tuple(lps if s is None else s), []).append(h)
+        spans_ref = [(s, g, None) for s, g in ref_spans]
+        self.groups = []
+        for box in sorted(groups):
+            lay = L.veda_plan(spans_ref + [(target[0], target[1], box)], seq_len, budgets[0], budgets[1])
+            hs = groups[box]
+            n = len(hs)
+            dev = self.device
+            g = dict(box=box, heads_list=hs, layout=lay,
+                     heads=torch.tensor(hs, dtype=torch.int32, device=dev),
+                     q_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
+                     k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
+                     v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
+                     feats_q=torch.empty(n, lay.n_video, 3 * dim, dtype=torch.float32, device=dev),
+                     feats_k=torch.empty(n, lay.n_video, 3 * dim, dtype=torch.float32, device=dev),
+                     workspace=torch.empty(L.veda_score_workspace_bytes(lay, n, dim) // 4, dtype=torch.float32,
+                                           device=dev),
+                     scores=torch.empty(n, lay.n_video, lay.n_video, dtype=torch.float32, device=dev),
+                     kept_idx=torch.empty(n, lay.n_video, lay.max_kept, dtype=torch.int32, device=dev),
+                     kept_cnt=torch.empty(n, lay.n_video, dtype=torch.int32, device=dev))
+            self.groups.append(g)
+        self.launches = self.LAUNCHES_PER_GROUP * len(self.groups)
+
+    def set_projections(self, proj_q, proj_k):
+        """proj_q, proj_k: fp32 [H, 3D, D] (any device); each group keeps its heads' slices on device."""
+        for g in self.groups:
+            idx = torch.tensor(g["heads_list"], dtype=torch.long)
+            g["proj_q"] = proj_q.index_select(0, idx).to(self.device, torch.float32).contiguous()
+            g["proj_k"] = proj_k.index_select(0, idx).to(self.device, torch.float32).contiguous()
+
+    def kept_tiles(self):
+        """Total kept (video query tile, key tile) pairs of the last forward, per the page's ``kept``."""
+        return sum(int(g["kept_cnt"].sum()) - g["layout"].n_global_ok * g["kept_cnt"].numel() for g in self.groups)
+
+    def work_tiles(self):
+        """The page's ``work`` counter (kept video pairs + dense global rows and columns), all groups."""
+        total = 0
+        for g in self.groups:
+            lay = g["layout"]
+            n = len(g["heads_list"])
+            kept_video = int(g["kept_cnt"].sum()) - lay.n_global_ok * n * lay.n_video
+            total += kept_video + n * lay.n_global * (lay.n_tiles + lay.n_video)
+        return total
+
+    def attended_tile_pairs(self):
+        """Tile pairs the attend kernels process: kept lists of video rows + dense lists of global rows."""
+        total = 0
+        for g in self.groups:
+            lay = g["layout"]
+            total += int(g["kept_cnt"].sum()) + len(g["heads_list"]) * lay.n_global * lay.n_kv_ok
+        return total
+
+    def forward(self, q, k, v, out, stream=None):
+        """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten."""
+        for g in self.groups:
+            lay = g["layout"]
+            L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], stream)
+            L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], stream)
+            L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"],
+                         stream)
+            L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], stream)
+            L.veda_gather(lay, v, g["heads"], g["v_t"], None, stream)
+            L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], stream)
+        return out

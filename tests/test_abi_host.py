@@ -1,0 +1,135 @@
+"""CPU checks of the C ABI: the library loads and exports every declared symbol, and the host planner
+(veda_plan and friends, no GPU needed) agrees bit for bit with the oracle."""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import veda_synth as V
+from learned_block_sparse_tile_b200 import _lib as L
+from learned_block_sparse_tile_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "veda.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(veda_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    lib = L.lib()
+    syms = declared_symbols()
+    assert len(syms) >= 14
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) == set(L.EXPORTS)
+
+
+def _plan_both(spans_o, seq_len, gen, ref):
+    lay_o = O.build_layout(spans_o, seq_len)
+    lay_c = L.veda_plan([(s, g, b) for s, g, b in spans_o], seq_len, gen, ref)
+    return lay_o, lay_c
+
+
+def _check_plan(spans_o, seq_len, gen, ref):
+    lay_o, lay_c = _plan_both(spans_o, seq_len, gen, ref)
+    perm, vc, allowed = L.veda_layout_export(lay_c)
+    assert np.array_equal(perm, lay_o.perm)
+    assert np.array_equal(vc, lay_o.valid_count)
+    assert (lay_c.n_video, lay_c.n_ref, lay_c.n_global) == (lay_o.n_video, lay_o.n_ref, lay_o.n_global)
+    blocks = O.column_blocks(lay_o, gen, ref)
+    assert len(blocks) == len(lay_c.blocks)
+    for b, blk in enumerate(blocks):
+        start, stop, budget, real = blk
+        cb = lay_c.blocks[b]
+        assert (cb[0], cb[1], cb[2]) == (start, stop, O.keeps_all(budget))
+        assert np.array_equal(allowed[b], O.allowed_per_row(lay_o, blk))
+        if not O.keeps_all(budget):
+            rb = O.row_budget(budget, real, stop - start)
+            lo, hi, frac = O.split_budget(rb, stop - start)
+            assert cb[6] == rb and (cb[3], cb[4]) == (lo, hi) and cb[5] == frac  # bit for bit
+    # an upper bound on every row's kept count, and the page's own bound (non-empty tiles)
+    assert lay_c.max_kept <= lay_o.widest
+    return lay_o, lay_c
+
+
+@pytest.mark.parametrize("name", ["tiny", "padded_tiny", "small_mixed", "small_dense", "small_d128", "single",
+                                  "mixed", "long", "sweep_tiles24", "sweep_r025", "sweep_r050", "sweep_dense"])
+def test_plan_matches_oracle_on_workloads(name):
+    wl = V.workload(name)
+    lps = O.least_padding_shape(wl.target[1])
+    tile_refs = not O.keeps_all(wl.reference)
+    for shape, _heads in V.head_groups(wl, lambda _: lps):
+        spans = O.veda.layer_spans(wl.ref_spans, (wl.target[0], wl.target[1], shape), tile_refs)
+        _check_plan(spans, wl.seq_len, wl.generated, wl.reference)
+
+
+def test_untiled_references_become_global():
+    wl = V.workload("small_mixed")
+    spans_c = [(s, g, None) for s, g in wl.ref_spans] + [(wl.target[0], wl.target[1], (2, 8, 8))]
+    lay_c = L.veda_plan(spans_c, wl.seq_len, (0.3, None), (1.0, None))
+    lay_o = O.build_layout([(wl.target[0], wl.target[1], (2, 8, 8))], wl.seq_len)
+    perm, vc, _ = L.veda_layout_export(lay_c)
+    assert lay_c.n_ref == 0 and np.array_equal(perm, lay_o.perm)
+
+
+def test_least_padding_box_matches_oracle():
+    rng = np.random.default_rng(0)
+    grids = [tuple(int(x) for x in rng.integers(1, 90, 3)) for _ in range(300)]
+    grids += [(26, 48, 84), (61, 45, 80), (1, 48, 84), (8, 16, 16), (1, 1, 1), (300, 2, 1)]
+    for g in grids:
+        assert L.veda_least_padding_box(g) == O.least_padding_shape(g), g
+
+
+def test_budget_split_sweep_bit_exact():
+    # many grids and budgets: the library's (k_lo, k_hi, frac, row budget) equal the oracle's bit for bit
+    rng = np.random.default_rng(1)
+    for _ in range(120):
+        grid = tuple(int(x) for x in rng.integers(1, 40, 3))
+        shape = O.tile_shapes()[int(rng.integers(0, 36))]
+        start = int(rng.integers(0, 300))
+        seq = start + grid[0] * grid[1] * grid[2] + int(rng.integers(0, 300))
+        if rng.random() < 0.5:
+            gen = (float(rng.choice([0.05, 0.1, 0.25, 0.3, 0.5, 0.75, 0.99, 1.0, 1.5, 0.001, 1 / 3])), None)
+        else:
+            gen = (None, int(rng.integers(0, 60)))
+        _check_plan([(start, grid, shape)], seq, gen, (1.0, None))
+
+
+def test_plan_errors():
+    with pytest.raises(L.VedaError) as e:
+        L.veda_plan([], 10, (0.1, None), (1.0, None))
+    assert e.value.code == L.VEDA_ERR_INVALID
+    for bad_budget in [(0.1, 3), (None, None), (-0.5, None)]:
+        with pytest.raises(L.VedaError):
+            L.veda_plan([(0, (1, 8, 16), None)], 128, bad_budget, (1.0, None))
+    with pytest.raises(L.VedaError):  # overlap
+        L.veda_plan([(0, (1, 8, 16), None), (100, (1, 8, 16), None)], 400, (0.1, None), (0.5, None))
+    with pytest.raises(L.VedaError):  # past the end
+        L.veda_plan([(10, (1, 8, 16), None)], 100, (0.1, None), (1.0, None))
+    with pytest.raises(L.VedaError):  # not a power-of-two box of 128
+        L.veda_plan([(0, (1, 8, 16), (1, 8, 15))], 128, (0.1, None), (1.0, None))
+    assert "overlaps" in L.veda_last_error() or L.veda_last_error() != ""
+
+
+def test_work_fraction_of_mixed_geometry():
+    # the library's per-row budgets reproduce the page's work counter on the mixed workload (10.85-11.07%)
+    wl = V.workload("mixed")
+    for box in [(1, 8, 16), (8, 4, 4), (2, 16, 4)]:
+        lay = L.veda_plan([(512, (1, 48, 84), None), (wl.target[0], wl.target[1], box)], wl.seq_len,
+                          wl.generated, wl.reference)
+        _, _, allowed = L.veda_layout_export(lay)
+        kept = int(allowed.sum())
+        work = kept + lay.n_global * (lay.n_tiles + lay.n_video)
+        frac = work / (wl.seq_len / 128) ** 2
+        assert 0.105 < frac < 0.112

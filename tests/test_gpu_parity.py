@@ -1,0 +1,152 @@
+"""GPU parity of every stage against the CPU oracle on small workloads (several tiles, ragged tails,
+padding, global rows, references, per-head boxes, head_dim 64 and 128). Calls go through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from learned_block_sparse_tile_b200 import _lib as L
+from learned_block_sparse_tile_b200 import build as B
+
+from gpu_util import (ATT_MAX_ABS, ATT_MEAN_ABS, POOL_ABS, POOL_REL, SCORE_REL, Case, attention_error,
+                      compare_lists, f32, gpu_lists, oracle_kept)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny", "padded_tiny", "small_mixed", "small_dense", "small_d128"]
+_cases = {}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+    L.veda_device_check()
+
+
+def case(name):
+    if name not in _cases:
+        _cases[name] = Case(name)
+    return _cases[name]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_stages_match_oracle(name):
+    c = case(name)
+    wl = c.wl
+    out = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    want_out = np.full((wl.seq_len, wl.heads, wl.dim), np.nan)
+    q, k, v = f32(c.q), f32(c.k), f32(c.v)
+    for box, heads in c.groups:
+        res = c.run_group(box, heads, out)
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        # gather: bit exact, head-major
+        for key, x in (("q_t", q), ("k_t", k), ("v_t", v)):
+            got = f32(res[key]).transpose(1, 0, 2)
+            assert np.array_equal(got, O.gather(x, lay_o, heads)), key
+        # pool: max/min exact, mean to fp32 rounding
+        for key, x in (("fq", q), ("fk", k)):
+            want = O.pool(O.gather(x, lay_o, heads), lay_o)
+            got = f32(res[key]).astype(np.float64)
+            D = wl.dim
+            assert np.array_equal(got[..., D:], want[..., D:]), key
+            assert np.all(np.abs(got[..., :D] - want[..., :D]) <= POOL_ABS + POOL_REL * np.abs(want[..., :D])), key
+        # score: on the GPU's own features, against float64 logits
+        fq, fk = f32(res["fq"]), f32(res["fk"])
+        want_s = O.logits(fq, fk, f32(c.pq[heads]), f32(c.pk[heads]))
+        got_s = f32(res["scores"])
+        for h in range(len(heads)):
+            assert np.abs(got_s[h] - want_s[h]).max() <= SCORE_REL * np.abs(want_s[h]).max()
+        # select: bit exact on identical scores
+        blocks = O.column_blocks(lay_o, wl.generated, wl.reference)
+        kept, mask = oracle_kept(lay_o, got_s, blocks)
+        compare_lists(res, mask, lay_o)
+        # attend: the oracle on the same kept sets
+        qt, kt, vt = (O.gather(x, lay_o, heads) for x in (q, k, v))
+        o_t = O.attend_tiles(qt, kt, vt, lay_o, lambda hh, i: np.flatnonzero(mask[hh, i]))
+        O.scatter(want_out, o_t, lay_o, heads)
+    got = f32(out)
+    assert not np.isnan(want_out).any()
+    mx, mean = attention_error(got, want_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+
+
+def test_keeps_all_equals_dense_attention():
+    c = case("small_dense")
+    wl = c.wl
+    out = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    for box, heads in c.groups:
+        c.run_group(box, heads, out)
+    want = O.dense_attention(f32(c.q), f32(c.k), f32(c.v))
+    mx, mean = attention_error(f32(out), want)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+
+
+def test_select_on_adversarial_scores():
+    # ties, NaN, -inf and +inf scores through the C ABI: lists equal the oracle's bit for bit
+    c = case("small_mixed")
+    wl = c.wl
+    box, heads = c.groups[0]
+    res = c.run_group(box, heads)
+    lay = res["layout"]
+    lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+    rng = np.random.default_rng(5)
+    s = np.round(rng.standard_normal((len(heads), lay.n_video, lay.n_video)) * 2).astype(np.float32)
+    s[0, 1, :5] = np.nan
+    s[0, 2, 3] = np.inf
+    s[0, 3, 4:9] = -np.inf
+    s[-1, :, 0] = 3.0
+    scores = torch.from_numpy(s).cuda()
+    L.veda_select(lay, scores, res["kept_idx"], res["kept_cnt"])
+    assert L.veda_sync_status() == L.VEDA_OK
+    _, mask = oracle_kept(lay_o, s, O.column_blocks(lay_o, wl.generated, wl.reference))
+    compare_lists(res, mask, lay_o)
+
+
+def test_empty_lists_give_zero_rows_and_head_order_is_free():
+    c = case("padded_tiny")
+    wl = c.wl
+    box, heads = c.groups[0]
+    res = c.run_group(box, list(reversed(heads)))  # heads [1, 0]
+    lay = res["layout"]
+    cnt = res["kept_cnt"].clone()
+    cnt[:, 0] = 0  # video query tile 0 keeps nothing
+    out = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    L.veda_attend(lay, res["q_t"], res["k_t"], res["v_t"], res["kept_idx"], cnt, out, res["heads"])
+    assert L.veda_sync_status() == L.VEDA_OK
+    perm, _, _ = L.veda_layout_export(lay)
+    rows0 = perm[:128][perm[:128] >= 0]
+    assert (f32(out)[rows0] == 0).all()
+    # every other row agrees with the normal run
+    other = np.setdiff1d(np.arange(wl.seq_len), rows0)
+    assert np.array_equal(f32(out)[other], f32(res["out"])[other])
+
+
+def test_malformed_lists_are_reported_not_faulted():
+    c = case("tiny")
+    box, heads = c.groups[0]
+    res = c.run_group(box, heads)
+    lay = res["layout"]
+    for mutate in ("range", "order", "count"):
+        idx, cnt = res["kept_idx"].clone(), res["kept_cnt"].clone()
+        if mutate == "range":
+            idx[0, 3, 1] = lay.n_tiles + 5
+        elif mutate == "order":
+            idx[1, 2, 2] = idx[1, 2, 1]
+        else:
+            cnt[0, 0] = lay.max_kept + 3
+        out = torch.zeros((c.wl.seq_len, c.wl.heads, c.wl.dim), dtype=torch.bfloat16, device="cuda")
+        L.veda_attend(lay, res["q_t"], res["k_t"], res["v_t"], idx, cnt, out, res["heads"])
+        assert L.veda_sync_status() == L.VEDA_ERR_BAD_LIST, mutate
+    assert L.veda_sync_status() == L.VEDA_OK  # the word was cleared
+
+
+def test_bad_arguments_rejected_on_host():
+    c = case("tiny")
+    box, heads = c.groups[0]
+    res = c.run_group(box, heads)
+    lay = res["layout"]
+    with pytest.raises(L.VedaError):  # D stride not 1
+        L.veda_gather(lay, c.dq.transpose(1, 2), res["heads"], res["q_t"], None)
+    with pytest.raises(L.VedaError):  # workspace too small
+        L.veda_score(lay, res["fq"], res["fk"], c.pq[heads].cuda(), c.pk[heads].cuda(),
+                     torch.empty(4, device="cuda"), res["scores"])

@@ -82,15 +82,43 @@ class VedaLayer:
             total += int(g["kept_cnt"].sum()) + len(g["heads_list"]) * lay.n_global * lay.n_kv_ok
         return total
 
-    def forward(self, q, k, v, out, stream=None):
-        """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten."""
+    def forward(self, q, k, v, out, stream=None, events=None):
+        """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten.
+
+        ``events``: optional dict; CUDA event pairs recorded around each stage on ``stream`` are appended
+        under the stage names gather_qk, score, select, gather_v and attend (the page's PhaseTimer)."""
+        st = stream if stream is not None else torch.cuda.current_stream()
+
+        def mark(name):
+            if events is None:
+                return None
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(st)
+            events.setdefault(name, []).append([e, None])
+            return name
+
+        def done(name):
+            if name is not None:
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(st)
+                events[name][-1][1] = e
+
         for g in self.groups:
             lay = g["layout"]
-            L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], stream)
-            L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], stream)
-            L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"],
-                         stream)
-            L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], stream)
-            L.veda_gather(lay, v, g["heads"], g["v_t"], None, stream)
-            L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], stream)
+            m = mark("gather_qk")
+            L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st)
+            L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st)
+            done(m)
+            m = mark("score")
+            L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"], st)
+            done(m)
+            m = mark("select")
+            L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], st)
+            done(m)
+            m = mark("gather_v")
+            L.veda_gather(lay, v, g["heads"], g["v_t"], None, st)
+            done(m)
+            m = mark("attend")
+            L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
+            done(m)
         return out

@@ -91,6 +91,9 @@ def workloads():
     w["sweep_fp8"] = Workload("sweep_fp8", 24, 128, 104832, (), (0, _GRID_104K), (None,) * 24,
                               _ratio(0.10), _DENSE, True, fp8_qk=True,
                               note="FP8 e4m3 Q/K with per-tile fp32 scales, ratio 0.10")
+    # the 104k-token layer with 4 heads: a profiling case that still exceeds L2 (322 MB of Q/K/V)
+    w["single_h4"] = Workload("single_h4", 4, 128, 104832, (), (0, _GRID_104K), (None,) * 4,
+                              _ratio(0.10), _DENSE, True, note="grid (26,48,84), 4 heads, ratio 0.10 (profiling)")
     # small cases that finish in seconds on the oracle and still span several tiles and a ragged tail
     w["padded_tiny"] = Workload("padded_tiny", 2, 64, 200 + 3 * 10 * 12, (), (200, (3, 10, 12)),
                                 ((2, 8, 8),) * 2, _ratio(0.5), _DENSE, True,

@@ -6,17 +6,25 @@
 // real rows are a prefix, so slot j of tile t is live iff j < valid_count[t]); a row that sees no key
 // gives 0. Then "tiles", scatter_: each real query slot goes to its packed row of the output.
 //
-// Design (one persistent CTA per SM, 192 threads, work items = (head, query tile)):
-//   warp 0      TMA producer: Q tile once per item, then K and V tiles of the item's kept list into a
-//               ring of STAGES stages (each TMA box is 128 rows x 128 bytes, 128-byte swizzle).
-//   warp 1      TMEM allocator and MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S buffers
-//               (128 fp32 columns each), O += P_j V_j into the TMEM O accumulator (D fp32 columns).
-//   warps 2-5   softmax: one thread per query row (its TMEM lane). Reads S_j, applies the key-slot mask,
-//               keeps a running max (rescaling O only when the max grows by more than 2^8, which keeps
-//               every P value below 256), writes P_j as bf16 into swizzled shared memory, and at the end
-//               of the item normalises O by the row sum and stores it to the packed output row.
-// Every wait is bounded (see ptx::mbar_wait); on expiry the CTA drains its in-flight copies and MMAs,
-// frees its TMEM and returns, and the host reads VEDA_ERR_TIMEOUT.
+// Design: one persistent CTA per SM, 384 threads, work items = (head, query tile), one item at a time.
+// The item's kept key tiles are split between two softmax warpgroups by parity, each with its own online
+// softmax state and its own O accumulator in TMEM; the two partial results are merged at the end of the
+// item. While one group computes its softmax the tensor core works on the other group's tiles.
+//   warp 0       TMA producer of Q (one buffer) and K (ring of 3); warp 2: TMA producer of V (ring of 2).
+//                Every box is 128 rows x 128 bytes with the 128-byte swizzle.
+//   warp 1       TMEM owner and MMA issuer (one thread): S_j = Q K_j^T (both operands in shared memory) into
+//                the S columns of group j%2, then O_(j%2) += P_j V_j with P read from TMEM where the group
+//                left it (the "TS" form) and V from shared memory. Issue order per item: S_0, S_1, then per
+//                tile PV_j followed by S_(j+2).
+//   warps 4-7    softmax group 0 (tiles 0, 2, 4, ...); warps 8-11 group 1 (tiles 1, 3, 5, ...). One thread
+//                per query row (its TMEM lane): masks key slots past the tile's real rows, keeps a running
+//                max (O is rescaled only when the max grows by more than 2^8, which bounds P by 256), and
+//                writes P as bf16 over its S columns. exp2 runs partly on the MUFU and partly as a polynomial
+//                on the FMA pipe. At the end of the item the groups exchange (max, sum) per row and each
+//                writes half of the output columns: (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / sum.
+// TMEM columns: S/P of group 0 [0,128), group 1 [128,256); O of group 0 [256, 256 + D), group 1 [384, 384 + D).
+// Every wait is bounded: on expiry the CTA drains its in-flight copies and MMAs, frees its TMEM and
+// returns, and the host reads VEDA_ERR_TIMEOUT.
 #pragma once
 
 #include <cuda.h>
@@ -27,6 +35,10 @@
 #include "ptx.cuh"
 
 namespace veda {
+
+// Of every 8 column pairs of a row, this many take exp2 on the FMA pipe (polynomial) and the rest on the
+// MUFU: 128 MUFU exp2 per row would cost 1024 cycles of one SMSP's MUFU per tile, more than the MMAs.
+constexpr int kPolyPairs = 3;
 
 constexpr int kErrTimeout = 1;
 constexpr int kErrBadList = 2;
@@ -51,21 +63,28 @@ struct AttendArgs {
 template <int D>
 struct AttendCfg {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-    static constexpr int kThreads = 192;
-    static constexpr int kTileBytes = 128 * D * 2;     // one Q, K or V tile (bf16)
-    static constexpr int kBoxes = D / 64;              // 64-column TMA boxes per tile
-    static constexpr int kPBytes = 128 * 128 * 2;      // P tile (bf16)
-    static constexpr int kStages = D == 128 ? 2 : 4;   // K/V ring depth
+    static constexpr int kWarps = 12;
+    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kTileBytes = 128 * D * 2;  // one Q, K or V tile (bf16)
+    static constexpr int kBoxes = D / 64;           // 64-column TMA boxes per tile
+    static constexpr int kKStages = 3;              // K ring depth
+    static constexpr int kVStages = 2;              // V ring depth
     static constexpr int kOffQ = 0;
-    static constexpr int kOffP = kOffQ + kTileBytes;
-    static constexpr int kOffKV = kOffP + kPBytes;     // stage s: K at kOffKV + 2s*tile, V right after
-    static constexpr int kOffBar = kOffKV + kStages * 2 * kTileBytes;
-    static constexpr int kBarBytes = 512;
-    static constexpr int kSmem = kOffBar + kBarBytes + 1024;  // + slack to align the base to 1024
-    static constexpr uint32_t kTmemCols = 512;         // S0 [0,128) S1 [128,256) O [256, 256 + D)
-    static constexpr uint32_t kColO = 256;
+    static constexpr int kOffK = kOffQ + kTileBytes;
+    static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+    static constexpr int kOffStats = kOffBar + 512;                     // [2 groups][128 rows] x (max, sum)
+    static constexpr int kSmem = kOffStats + 2 * 128 * 8 + 1024;        // + slack to align the base to 1024
+    static constexpr uint32_t kTmemCols = 512;  // S/P of group 0, S/P of group 1, O of group 0, O of group 1
     static constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, false, true);
+};
+
+struct AttendBars {
+    uint64_t q_full, q_empty;
+    uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t o_empty, merge, drain;
 };
 
 // Number of kept tiles of an item and its list. Warp-collective (all 32 lanes, same result in each).
@@ -106,8 +125,10 @@ __device__ __forceinline__ int item_tiles(const AttendArgs& a, int hh, int qt, c
     return n;
 }
 
+// Item order: the dense global query tiles first (they are the longest), then head-major video tiles,
+// so that neighbouring slots work on neighbouring query tiles of one head (shared K/V in L2).
 __device__ __forceinline__ void decode_item(const AttendArgs& a, int item, int* hh, int* qt) {
-    const int n_glob_items = a.n_heads * a.n_global;  // dense global rows first: they are the longest
+    const int n_glob_items = a.n_heads * a.n_global;
     if (item < n_glob_items) {
         *hh = item / a.n_global;
         *qt = a.n_video + item % a.n_global;
@@ -118,48 +139,43 @@ __device__ __forceinline__ void decode_item(const AttendArgs& a, int item, int* 
     }
 }
 
+
+// Tiles of an item that softmax group w handles: the item-local tiles j = w, w + 2, ...
+__device__ __forceinline__ int group_tiles(int n, int w) { return (n - w + 1) >> 1; }
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const AttendArgs a) {
     using C = AttendCfg<D>;
-    constexpr int S = C::kStages;
+    constexpr int KS = C::kKStages, VS = C::kVStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* q_full = bars + 0;
-    uint64_t* q_empty = bars + 1;
-    uint64_t* k_full = bars + 2;
-    uint64_t* v_full = k_full + S;
-    uint64_t* kv_empty = v_full + S;
-    uint64_t* s_full = kv_empty + S;   // [2]
-    uint64_t* s_empty = s_full + 2;    // [2]
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* o_done = p_full + 1;
-    uint64_t* o_empty = o_done + 1;
-    uint64_t* drain = o_empty + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    AttendBars& B = *reinterpret_cast<AttendBars*>(smem + C::kOffBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&B + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* kvalid = const_cast<int*>(abort_flag) + 1;  // [S]
+    float2* stats = reinterpret_cast<float2*>(smem + C::kOffStats);  // [2 groups][128 rows] (max, sum)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        ptx::mbar_init(q_full, 1);
-        ptx::mbar_init(q_empty, 1);
-        for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(k_full + s, 1);
-            ptx::mbar_init(v_full + s, 1);
-            ptx::mbar_init(kv_empty + s, 1);
+        ptx::mbar_init(&B.q_full, 1);
+        ptx::mbar_init(&B.q_empty, 1);
+        for (int i = 0; i < KS; ++i) {
+            ptx::mbar_init(&B.k_full[i], 1);
+            ptx::mbar_init(&B.k_empty[i], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(s_full + b, 1);
-            ptx::mbar_init(s_empty + b, 128);
+        for (int i = 0; i < VS; ++i) {
+            ptx::mbar_init(&B.v_full[i], 1);
+            ptx::mbar_init(&B.v_empty[i], 1);
         }
-        ptx::mbar_init(p_full, 128);
-        ptx::mbar_init(o_done, 1);
-        ptx::mbar_init(o_empty, 128);
-        ptx::mbar_init(drain, 1);
+        for (int w = 0; w < 2; ++w) {
+            ptx::mbar_init(&B.s_full[w], 1);
+            ptx::mbar_init(&B.p_full[w], 128);
+            ptx::mbar_init(&B.o_done[w], 1);
+        }
+        ptx::mbar_init(&B.o_empty, 256);
+        ptx::mbar_init(&B.merge, 256);
+        ptx::mbar_init(&B.drain, 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -174,54 +190,43 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = a.timeout_ns;
 
-    const uint32_t sm_q = ptx::smem_addr(smem + C::kOffQ);
-    const uint32_t sm_p = ptx::smem_addr(smem + C::kOffP);
-    const uint32_t sm_kv = ptx::smem_addr(smem + C::kOffKV);
-
-    if (warp == 0) {
-        // ------------------------------------------------------------------------------ producer
-        int g = 0, it_local = 0;
-        int last_use[S];
-        for (int s = 0; s < S; ++s) last_use[s] = -1;
-        int last_q = -1;
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------- producers: warp 0 Q and K, warp 2 V
+        const bool kq = warp == 0;
+        const int S = kq ? KS : VS;
         const uint64_t keep = ptx::policy_evict_last();
+        int issued_q = 0, issued = 0;  // copies issued so far (lane 0): Q tiles; K or V tiles
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
-            if (bad && lane == 0) atomicOr(a.err, kErrBadList);
+            if (kq && bad && lane == 0) atomicOr(a.err, kErrBadList);
             if (n == 0) continue;
             const int32_t row0 = int32_t(int64_t(hh) * a.n_slots);
-            if (lane == 0) {
-                if (ptx::mbar_wait(q_empty, (it_local & 1) ^ 1, abort_flag, tmo)) {
-                    ptx::mbar_arrive_expect_tx(q_full, C::kTileBytes);
-                    for (int b = 0; b < C::kBoxes; ++b)
-                        ptx::tma_load_2d(smem + C::kOffQ + b * 16384, &tm_q, b * 64, row0 + qt * 128, q_full);
-                    last_q = it_local;
-                }
+            if (kq && lane == 0 && ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo)) {
+                ptx::mbar_arrive_expect_tx(&B.q_full, C::kTileBytes);
+                for (int x = 0; x < C::kBoxes; ++x)
+                    ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * 64, row0 + qt * 128, &B.q_full);
+                ++issued_q;
             }
-            ++it_local;
             __syncwarp();
             if (*abort_flag) break;
             int mine = 0;
-            for (int j = 0; j < n; ++j, ++g) {
+            for (int j = 0; j < n; ++j) {
                 if ((j & 31) == 0) mine = (j + lane < n) ? __ldg(list + j + lane) : 0;
-                const int tile = __shfl_sync(0xffffffffu, mine, j & 31);
+                const int y = row0 + __shfl_sync(0xffffffffu, mine, j & 31) * 128;
                 if (lane == 0) {
-                    const int st = g % S, u = g / S;
-                    if (ptx::mbar_wait(kv_empty + st, (u & 1) ^ 1, abort_flag, tmo)) {
-                        kvalid[st] = __ldg(a.valid_count + tile);
-                        uint8_t* kd = smem + C::kOffKV + st * 2 * C::kTileBytes;
-                        ptx::mbar_arrive_expect_tx(k_full + st, C::kTileBytes);
-                        for (int b = 0; b < C::kBoxes; ++b)
-                            ptx::tma_load_2d_hint(kd + b * 16384, &tm_k, b * 64, row0 + tile * 128, k_full + st, keep);
-                        ptx::mbar_arrive_expect_tx(v_full + st, C::kTileBytes);
-                        for (int b = 0; b < C::kBoxes; ++b)
-                            ptx::tma_load_2d_hint(kd + C::kTileBytes + b * 16384, &tm_v, b * 64, row0 + tile * 128,
-                                                  v_full + st, keep);
-                        last_use[st] = u;
+                    const int st = issued % S, u = issued / S;
+                    uint64_t* empty = kq ? &B.k_empty[st] : &B.v_empty[st];
+                    uint64_t* full = kq ? &B.k_full[st] : &B.v_full[st];
+                    uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * C::kTileBytes;
+                    if (ptx::mbar_wait(empty, (u & 1) ^ 1, abort_flag, tmo)) {
+                        ptx::mbar_arrive_expect_tx(full, C::kTileBytes);
+                        for (int x = 0; x < C::kBoxes; ++x)
+                            ptx::tma_load_2d_hint(dst + x * 16384, kq ? &tm_k : &tm_v, x * 64, y, full, keep);
+                        ++issued;
                     }
                 }
                 __syncwarp();
@@ -230,18 +235,18 @@ __global__ void __launch_bounds__(192, 1)
             if (*abort_flag) break;
         }
         if (*abort_flag && lane == 0) {
-            // let every copy already issued land before the CTA releases its shared memory
+            // every copy already issued must land before the CTA releases its shared memory
             volatile int never = 0;
-            for (int s = 0; s < S; ++s)
-                if (last_use[s] >= 0) {
-                    ptx::mbar_wait(k_full + s, last_use[s] & 1, &never, tmo);
-                    ptx::mbar_wait(v_full + s, last_use[s] & 1, &never, tmo);
-                }
-            if (last_q >= 0) ptx::mbar_wait(q_full, last_q & 1, &never, tmo);
+            for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
+                ptx::mbar_wait(kq ? &B.k_full[k % KS] : &B.v_full[k % VS], (k / S) & 1, &never, tmo);
+            if (kq && issued_q > 0) ptx::mbar_wait(&B.q_full, (issued_q - 1) & 1, &never, tmo);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------------------------ MMA issuer
-        int g = 0, sc = 0, pc = 0, it_local = 0, o_uses = 0;
+        // ------------------------------------------------------------- MMA issuer (one thread)
+        // Per item: S_0 and S_1, then for each tile j: O_(j%2) += P_j V_j, then S_(j+2). S_j lands in S
+        // buffer j%2, which softmax group j%2 turns into P_j in place.
+        int it = 0, t = 0;      // items with tiles so far; tiles so far (ring positions)
+        int pu[2] = {0, 0};     // tiles each group has had so far (barrier phases)
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
@@ -250,68 +255,71 @@ __global__ void __launch_bounds__(192, 1)
             const int n = item_tiles(a, hh, qt, &list, &bad);
             if (n == 0) continue;
             if (lane == 0) {
-                bool ok = ptx::mbar_wait(q_full, it_local & 1, abort_flag, tmo);
-                ptx::tc_fence_after();
-                for (int j = 0; ok && j <= n; ++j) {
-                    if (j < n) {
-                        const int st = (g + j) % S, u = (g + j) / S, b = sc & 1;
-                        ok = ptx::mbar_wait(k_full + st, u & 1, abort_flag, tmo) &&
-                             ptx::mbar_wait(s_empty + b, ((sc >> 1) & 1) ^ 1, abort_flag, tmo);
+                const uint32_t q0 = ptx::smem_addr(smem + C::kOffQ);
+                bool ok = ptx::mbar_wait(&B.q_full, it & 1, abort_flag, tmo);
+                for (int j = 0; ok && j < n + 2; ++j) {
+                    if (j >= 2) {
+                        // O_w += P V for tile jj = j - 2
+                        const int jj = j - 2, w = jj & 1, idx = pu[w] + (jj >> 1), tv = t + jj, sv = tv % VS;
+                        ok = ptx::mbar_wait(&B.p_full[w], idx & 1, abort_flag, tmo) &&
+                             ptx::mbar_wait(&B.v_full[sv], (tv / VS) & 1, abort_flag, tmo) &&
+                             (jj > 0 || ptx::mbar_wait(&B.o_empty, (it & 1) ^ 1, abort_flag, tmo));
                         if (!ok) break;
                         ptx::tc_fence_after();
-                        const uint32_t kbase = sm_kv + st * 2 * C::kTileBytes;
+                        const uint32_t v0 = ptx::smem_addr(smem + C::kOffV + sv * C::kTileBytes);
+                        const uint32_t o = tmem + 256 + 128 * w, p = tmem + 128 * w;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            ptx::mma_bf16_ts(o, p + kk * 8, ptx::smem_desc_sw128(v0 + kk * 2048, 16384, 1024), C::kIdescPV,
+                                             (jj >= 2 || kk > 0) ? 1u : 0u);
+                        ptx::mma_commit(&B.o_done[w]);
+                        ptx::mma_commit(&B.v_empty[sv]);
+                    }
+                    if (j < n) {
+                        // S_j = Q K_j^T into S buffer j%2
+                        const int w = j & 1, tk = t + j, st = tk % KS;
+                        ok = ptx::mbar_wait(&B.k_full[st], (tk / KS) & 1, abort_flag, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        const uint32_t k0 = ptx::smem_addr(smem + C::kOffK + st * C::kTileBytes);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                            ptx::mma_bf16_ss(tmem + b * 128, ptx::smem_desc_sw128(sm_q + off, 16, 1024),
-                                             ptx::smem_desc_sw128(kbase + off, 16, 1024), C::kIdescS, kk > 0);
+                            ptx::mma_bf16_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
+                                             ptx::smem_desc_sw128(k0 + off, 16, 1024), C::kIdescS, kk > 0);
                         }
-                        ptx::mma_commit(s_full + b);
-                        ++sc;
-                        if (j == n - 1) ptx::mma_commit(q_empty);
-                    }
-                    if (j >= 1) {
-                        const int jj = j - 1, st = (g + jj) % S, u = (g + jj) / S;
-                        ok = ptx::mbar_wait(v_full + st, u & 1, abort_flag, tmo) &&
-                             ptx::mbar_wait(p_full, pc & 1, abort_flag, tmo);
-                        if (ok && jj == 0) {
-                            ok = ptx::mbar_wait(o_empty, (o_uses & 1) ^ 1, abort_flag, tmo);
-                            ++o_uses;
-                        }
-                        if (!ok) break;
-                        ptx::tc_fence_after();
-                        const uint32_t vbase = sm_kv + st * 2 * C::kTileBytes + C::kTileBytes;
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t poff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                            ptx::mma_bf16_ss(tmem + C::kColO, ptx::smem_desc_sw128(sm_p + poff, 16, 1024),
-                                             ptx::smem_desc_sw128(vbase + kk * 2048, 16384, 1024), C::kIdescPV,
-                                             (jj > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        ptx::mma_commit(o_done);
-                        ptx::mma_commit(kv_empty + st);
-                        ++pc;
+                        ptx::mma_commit(&B.s_full[w]);
+                        ptx::mma_commit(&B.k_empty[st]);
+                        if (j == n - 1) ptx::mma_commit(&B.q_empty);
                     }
                 }
             }
-            g += n;
-            ++it_local;
+            t += n;
+            pu[0] += group_tiles(n, 0);
+            pu[1] += group_tiles(n, 1);
+            ++it;
             __syncwarp();
             if (*abort_flag) break;
         }
         if (lane == 0) {
             // every MMA issued so far must finish before the TMEM is released
             volatile int never = 0;
-            ptx::mma_commit(drain);
-            ptx::mbar_wait(drain, 0, &never, tmo);
+            ptx::mma_commit(&B.drain);
+            ptx::mbar_wait(&B.drain, 0, &never, tmo);
         }
-    } else {
-        // ------------------------------------------------------------------------------ softmax
-        const int q4 = warp & 3;
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------- softmax groups (warps 4-7, 8-11)
+        const int w = (warp - 4) >> 2;  // group: item-local tiles j with j % 2 == w
+        const int q4 = warp & 3;        // TMEM lane quarter this warp may access
         const int row = q4 * 32 + lane;
         const uint32_t lane_base = uint32_t(q4 * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + 128 * w;        // S / P of this group
+        const uint32_t t_o = tmem + lane_base + 256 + 128 * w;  // O of this group
+        const uint32_t t_o0 = tmem + lane_base + 256;
         const float sl2 = a.scale_log2;
-        int g = 0, sc = 0, pc = 0;
+        const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
+        int cu[2] = {0, 0};  // tiles each group has had so far (barrier phases)
+        int it = 0;
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
@@ -320,125 +328,160 @@ __global__ void __launch_bounds__(192, 1)
             const int n = item_tiles(a, hh, qt, &list, &bad);
             const int head = __ldg(a.heads + hh);
             const bool head_ok = head >= 0 && head < a.h_total;
-            if (!head_ok && threadIdx.x == 64) atomicOr(a.err, 4);
+            if (!head_ok && threadIdx.x == 128) atomicOr(a.err, 4);
             const int prow = head_ok ? __ldg(a.perm + int64_t(qt) * 128 + row) : -1;
-            __nv_bfloat16* dst = a.out + int64_t(prow < 0 ? 0 : prow) * a.out_s0 + int64_t(head_ok ? head : 0) * a.out_s1;
+            // this group writes output columns [w D/2, (w + 1) D/2) of its rows
+            __nv_bfloat16* dst = a.out + int64_t(prow < 0 ? 0 : prow) * a.out_s0 +
+                                 int64_t(head_ok ? head : 0) * a.out_s1 + w * (D / 2);
             if (n == 0) {
                 if (prow >= 0) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
+                    for (int c = 0; c < D / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
                 }
                 continue;
             }
-            float m_ref = -INFINITY, l = 0.f;
+            const int nw = group_tiles(n, w);
+            float m_ref = -INFINITY;
+            uint64_t lsum = ptx::f2_pack(0.f, 0.f);
             bool ok = true;
-            for (int j = 0; j < n; ++j) {
-                const int b = sc & 1;
-                ok = ptx::mbar_wait(s_full + b, (sc >> 1) & 1, abort_flag, tmo);
+            int my_vc = 128;
+            for (int k = 0; k < nw; ++k) {
+                if ((k & 31) == 0) {
+                    const int jj = 2 * (k + lane) + w;
+                    my_vc = jj < n ? __ldg(a.valid_count + __ldg(list + jj)) : 128;
+                }
+                const int vc = __shfl_sync(0xffffffffu, my_vc, k & 31);
+                const int idx = cu[w] + k;
+                ok = ptx::mbar_wait(&B.s_full[w], idx & 1, abort_flag, tmo);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 uint32_t s[128];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(s + 32 * i);
-                    ptx::tmem_ld32(tmem + lane_base + b * 128 + 32 * i, chunk);
-                }
+                for (int i = 0; i < 4; ++i)
+                    ptx::tmem_ld32(t_s + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(s + 32 * i));
                 ptx::tmem_wait_ld();
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(s_empty + b);
-                ++sc;
-                const int st = (g + j) % S, u = (g + j) / S;
-                ok = ptx::mbar_wait(k_full + st, u & 1, abort_flag, tmo);  // already complete: orders kvalid
-                if (!ok) break;
-                const int vc = kvalid[st];
-                float mx = -INFINITY;
-                if (vc >= 128) {
-#pragma unroll
-                    for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-                } else {
+                if (vc < 128) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
-                        if (c < vc) mx = fmaxf(mx, __uint_as_float(s[c]));
+                        if (c >= vc) s[c] = __float_as_uint(-INFINITY);
                 }
+                // row max: 8 independent chains of 3-input maxima
+                float mx8[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(__uint_as_float(s[q]), __uint_as_float(s[8 + q]));
+#pragma unroll
+                for (int c = 16; c < 128; c += 16) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        mx8[q] = ptx::max3(mx8[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
+                }
+                const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
+                                           fmaxf(mx8[6], mx8[7]));
                 const float m_new = mx * sl2;
                 const bool resc = m_new > m_ref + 8.0f;
                 float alpha = 1.f;
                 if (resc) {
                     alpha = ptx::ex2(m_ref - m_new);
-                    l *= alpha;
+                    lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
                     m_ref = m_new;
                 }
-                const float neg = -m_ref;
-                float rs = 0.f;
+                const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
+                const uint64_t negm2 = ptx::f2_pack(negm, negm);
+                uint64_t acc[4] = {ptx::f2_pack(0.f, 0.f), ptx::f2_pack(0.f, 0.f), ptx::f2_pack(0.f, 0.f),
+                                   ptx::f2_pack(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < 128; c += 2) {
-                    float p0 = ptx::ex2(fmaf(__uint_as_float(s[c]), sl2, neg));
-                    float p1 = ptx::ex2(fmaf(__uint_as_float(s[c + 1]), sl2, neg));
-                    if (vc < 128) {
-                        p0 = c < vc ? p0 : 0.f;
-                        p1 = c + 1 < vc ? p1 : 0.f;
+                    const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2, negm2);
+                    float p0, p1;
+                    if (((c >> 1) & 7) < kPolyPairs) {  // this pair on the FMA pipe
+                        ptx::f2_unpack(ptx::f2_exp2_poly(x), p0, p1);
+                    } else {  // this pair on the MUFU
+                        float x0, x1;
+                        ptx::f2_unpack(x, x0, x1);
+                        p0 = ptx::ex2(x0);
+                        p1 = ptx::ex2(x1);
                     }
-                    rs += p0 + p1;
+                    acc[(c >> 1) & 3] = ptx::f2_add(acc[(c >> 1) & 3], ptx::f2_pack(p0, p1));
                     s[c >> 1] = ptx::pack_bf16(p0, p1);
                 }
-                l += rs;
-                if (j > 0) {
-                    ok = ptx::mbar_wait(o_done, pc & 1, abort_flag, tmo);
-                    ++pc;
+                lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])));
+                if (k > 0) {
+                    // the PV of this group's previous tile must finish before O is rescaled or reused
+                    ok = ptx::mbar_wait(&B.o_done[w], (idx - 1) & 1, abort_flag, tmo);
                     if (!ok) break;
                     ptx::tc_fence_after();
                     if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
                         for (int i = 0; i < D / 32; ++i) {
                             uint32_t o[32];
-                            ptx::tmem_ld32(tmem + lane_base + C::kColO + 32 * i, o);
+                            ptx::tmem_ld32(t_o + 32 * i, o);
                             ptx::tmem_wait_ld();
 #pragma unroll
                             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                            ptx::tmem_st32(tmem + lane_base + C::kColO + 32 * i, o);
+                            ptx::tmem_st32(t_o + 32 * i, o);
                         }
-                        ptx::tmem_wait_st();
                     }
                 }
-                // P row -> two 64-key swizzle atoms (128 rows x 128 bytes each), K-major
-                const uint32_t rbase = sm_p + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-                for (int c16 = 0; c16 < 16; ++c16) {
-                    const uint32_t addr = rbase + (c16 >> 3) * 16384 + (((c16 & 7) ^ (row & 7)) << 4);
-                    ptx::st_shared_v4(addr, s[c16 * 4 + 0], s[c16 * 4 + 1], s[c16 * 4 + 2], s[c16 * 4 + 3]);
-                }
-                ptx::fence_proxy_async_smem();
+                // P (bf16 pairs) over the first 64 S columns: the A operand of O += P V
+                ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
+                ptx::tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
+                ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(p_full);
+                ptx::mbar_arrive(&B.p_full[w]);
             }
-            g += n;
             if (!ok) break;
-            // epilogue: O / l -> bf16 -> packed output row
-            ok = ptx::mbar_wait(o_done, pc & 1, abort_flag, tmo);
-            ++pc;
+            // both groups' last PVs of this item must be complete before either accumulator is read. This
+            // group's own barrier first: it has followed it phase by phase, and once its last PV is done every
+            // earlier MMA is too, so the other group's barrier is at most one phase short of its last PV
+            // (a parity wait is only meaningful within one phase).
+            const int n0 = group_tiles(n, 0), n1 = group_tiles(n, 1);
+            const int nmine = w ? n1 : n0, nother = w ? n0 : n1;
+            ok = (nmine == 0 || ptx::mbar_wait(&B.o_done[w], (cu[w] + nmine - 1) & 1, abort_flag, tmo)) &&
+                 (nother == 0 || ptx::mbar_wait(&B.o_done[w ^ 1], (cu[w ^ 1] + nother - 1) & 1, abort_flag, tmo));
+            cu[0] += n0;
+            cu[1] += n1;
             if (!ok) break;
+            // merge the two groups: exchange (max, sum) per row through shared memory
+            float l0, l1;
+            ptx::f2_unpack(lsum, l0, l1);
+            stats[w * 128 + row] = make_float2(m_ref, l0 + l1);
+            ptx::mbar_arrive(&B.merge);
+            ok = ptx::mbar_wait(&B.merge, it & 1, abort_flag, tmo);
+            ++it;
+            if (!ok) break;
+            const float2 st0 = stats[row], st1 = stats[128 + row];
+            const float m = fmaxf(st0.x, st1.x);
+            const float a0 = st0.y > 0.f ? ptx::ex2(st0.x - m) : 0.f;
+            const float a1 = st1.y > 0.f ? ptx::ex2(st1.x - m) : 0.f;
+            const float den = a0 * st0.y + a1 * st1.y;
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            const float s0 = a0 * inv, s1 = a1 * inv;
             ptx::tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tmem + lane_base + C::kColO + 32 * i, o);
+            for (int i = 0; i < D / 64; ++i) {
+                const uint32_t col = w * (D / 2) + 32 * i;
+                uint32_t o0[32], o1[32];
+                ptx::tmem_ld32(t_o0 + col, o0);
+                ptx::tmem_ld32(t_o0 + 128 + col, o1);
                 ptx::tmem_wait_ld();
-                if (i == D / 32 - 1) {
+                if (i == D / 64 - 1) {
                     ptx::tc_fence_before();
-                    ptx::mbar_arrive(o_empty);
+                    ptx::mbar_arrive(&B.o_empty);
                 }
                 if (prow >= 0) {
                     uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * i);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        uint4 w;
-                        w.x = ptx::pack_bf16(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-                        w.y = ptx::pack_bf16(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-                        w.z = ptx::pack_bf16(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-                        w.w = ptx::pack_bf16(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-                        d4[c] = w;
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float x0 = s0 != 0.f ? __uint_as_float(o0[8 * c + e]) * s0 : 0.f;
+                            const float x1 = s1 != 0.f ? __uint_as_float(o1[8 * c + e]) * s1 : 0.f;
+                            v[e] = x0 + x1;
+                        }
+                        d4[c] = make_uint4(ptx::pack_bf16(v[0], v[1]), ptx::pack_bf16(v[2], v[3]),
+                                           ptx::pack_bf16(v[4], v[5]), ptx::pack_bf16(v[6], v[7]));
                     }
                 }
             }

@@ -49,6 +49,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// Non-blocking probe of the same condition.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Waits until the phase of parity `parity` of `bar` has completed. Gives up (returns false) when
 // `*abort` becomes non-zero or after `timeout_ns`; on a timeout it raises `*abort` itself.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
@@ -137,6 +150,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, one CTA. A (M x K, K-major) sits in TMEM lanes 0..M-1,
+// two 16-bit elements per 32-bit column.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 async operation this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -200,6 +225,60 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
 }
 
 // ---------------------------------------------------------------------------------------- math
+
+// Packed pairs of fp32 (sm_100 f32x2 pipe ops): lo in bits 0-31, hi in bits 32-63.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// 2^x for a pair of fp32 values on the FMA pipe (x <= 126; inputs below -126 are taken as -126, giving
+// ~1e-38). Cody-Waite range reduction x = n + f with n = round(x) via the 1.5 * 2^23 rounding constant,
+// then 2^f ~ c0 + f (c1 + f (c2 + f c3)) on [-1/2, 1/2] (coefficients from gen_exp2_poly.py, max relative
+// error 7.6e-5), and 2^n applied by adding n to the exponent field.
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+    const uint64_t r = f2_add(x, magic);  // low mantissa bits hold round(x)
+    const uint64_t nf = f2_add(r, f2_pack(-12582912.f, -12582912.f));
+    const uint64_t f = f2_fma(nf, f2_pack(-1.f, -1.f), x);
+    uint64_t p = f2_fma(f2_pack(0.05517049878835678f, 0.05517049878835678f), f,
+                        f2_pack(0.24260851740837097f, 0.24260851740837097f));
+    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, f, f2_pack(0.9999282360076904f, 0.9999282360076904f));
+    uint32_t p0, p1, r0, r1;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(r));
+    uint64_t out;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(out) : "r"(r0 * 8388608u + p0), "r"(r1 * 8388608u + p1));
+    return out;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 __device__ __forceinline__ float ex2(float x) {
     float y;

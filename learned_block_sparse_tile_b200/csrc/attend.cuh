@@ -10,7 +10,7 @@
 // The item's kept key tiles are split between two softmax warpgroups by parity, each with its own online
 // softmax state and its own O accumulator in TMEM; the two partial results are merged at the end of the
 // item. While one group computes its softmax the tensor core works on the other group's tiles.
-//   warp 0       TMA producer of Q (one buffer) and K (ring of 3); warp 2: TMA producer of V (ring of 2).
+//   warp 0       TMA producer of Q (one buffer) and K (ring of 3); warp 2: TMA producer of V (ring of 3).
 //                Every box is 128 rows x 128 bytes with the 128-byte swizzle.
 //   warp 1       TMEM owner and MMA issuer (one thread): S_j = Q K_j^T (both operands in shared memory) into
 //                the S columns of group j%2, then O_(j%2) += P_j V_j with P read from TMEM where the group
@@ -42,6 +42,7 @@ constexpr int kPolyPairs = 3;
 
 constexpr int kErrTimeout = 1;
 constexpr int kErrBadList = 2;
+constexpr int kErrLayout = 8;  // shared memory base not 1024-byte aligned: the kernel did nothing
 
 struct AttendArgs {
     const int32_t* kept_idx;     // [n_heads, n_video, max_kept]
@@ -68,13 +69,16 @@ struct AttendCfg {
     static constexpr int kTileBytes = 128 * D * 2;  // one Q, K or V tile (bf16)
     static constexpr int kBoxes = D / 64;           // 64-column TMA boxes per tile
     static constexpr int kKStages = 3;              // K ring depth
-    static constexpr int kVStages = 2;              // V ring depth
-    static constexpr int kOffQ = 0;
+    static constexpr int kVStages = 3;              // V ring depth
+    // header (barriers, then the [2 groups][128 rows] (max, sum) exchange) first, then the 1024-aligned
+    // tiles; with a 1024-aligned dynamic base this fills the 227 KB a CTA may use at head_dim 128
+    static constexpr int kOffBar = 0;
+    static constexpr int kOffStats = 256;
+    static constexpr int kHeader = 3072;
+    static constexpr int kOffQ = kHeader;
     static constexpr int kOffK = kOffQ + kTileBytes;
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-    static constexpr int kOffStats = kOffBar + 512;                     // [2 groups][128 rows] x (max, sum)
-    static constexpr int kSmem = kOffStats + 2 * 128 * 8 + 1024;        // + slack to align the base to 1024
+    static constexpr int kSmem = kOffV + kVStages * kTileBytes;
     static constexpr uint32_t kTmemCols = 512;  // S/P of group 0, S/P of group 1, O of group 0, O of group 1
     static constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, false, true);
@@ -82,7 +86,7 @@ struct AttendCfg {
 
 struct AttendBars {
     uint64_t q_full, q_empty;
-    uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+    uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
     uint64_t s_full[2], p_full[2], o_done[2];
     uint64_t o_empty, merge, drain;
 };
@@ -149,8 +153,12 @@ __global__ void __launch_bounds__(384, 1)
                   const __grid_constant__ CUtensorMap tm_v, const AttendArgs a) {
     using C = AttendCfg<D>;
     constexpr int KS = C::kKStages, VS = C::kVStages;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw;
+    if ((ptx::smem_addr(smem) & 1023) != 0) {  // the swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
+        return;
+    }
     AttendBars& B = *reinterpret_cast<AttendBars*>(smem + C::kOffBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&B + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -272,8 +280,8 @@ __global__ void __launch_bounds__(384, 1)
                         for (int kk = 0; kk < 8; ++kk)
                             ptx::mma_bf16_ts(o, p + kk * 8, ptx::smem_desc_sw128(v0 + kk * 2048, 16384, 1024), C::kIdescPV,
                                              (jj >= 2 || kk > 0) ? 1u : 0u);
-                        ptx::mma_commit(&B.o_done[w]);
                         ptx::mma_commit(&B.v_empty[sv]);
+                        if (jj >= n - 2) ptx::mma_commit(&B.o_done[w]);  // the group's last tile of the item
                     }
                     if (j < n) {
                         // S_j = Q K_j^T into S buffer j%2
@@ -288,8 +296,7 @@ __global__ void __launch_bounds__(384, 1)
                             ptx::mma_bf16_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
                                              ptx::smem_desc_sw128(k0 + off, 16, 1024), C::kIdescS, kk > 0);
                         }
-                        ptx::mma_commit(&B.s_full[w]);
-                        ptx::mma_commit(&B.k_empty[st]);
+                        ptx::mma_commit(&B.s_full[w]);  // the softmax group also frees the K slot on it
                         if (j == n - 1) ptx::mma_commit(&B.q_empty);
                     }
                 }
@@ -319,7 +326,9 @@ __global__ void __launch_bounds__(384, 1)
         const float sl2 = a.scale_log2;
         const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
         int cu[2] = {0, 0};  // tiles each group has had so far (barrier phases)
-        int it = 0;
+        int it = 0, t = 0;   // items with tiles so far; tiles so far (K ring positions)
+        int od[2] = {0, 0};  // o_done phases: one per item in which the group had a tile
+        const bool releaser = (warp & 3) == 0 && lane == 0;  // one thread per group frees K slots
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
@@ -356,6 +365,10 @@ __global__ void __launch_bounds__(384, 1)
                 ok = ptx::mbar_wait(&B.s_full[w], idx & 1, abort_flag, tmo);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                // S of this tile is complete, so its K slot may be refilled. S of this group's tile was also
+                // issued after the PV of the group's previous tile, so that PV is complete as well: O may be
+                // rescaled and the P columns rewritten without another wait.
+                if (releaser) ptx::mbar_arrive(&B.k_empty[(t + 2 * k + w) % KS]);
                 uint32_t s[128];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
@@ -407,10 +420,6 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])));
                 if (k > 0) {
-                    // the PV of this group's previous tile must finish before O is rescaled or reused
-                    ok = ptx::mbar_wait(&B.o_done[w], (idx - 1) & 1, abort_flag, tmo);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
                     if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
                         for (int i = 0; i < D / 32; ++i) {
@@ -437,10 +446,13 @@ __global__ void __launch_bounds__(384, 1)
             // (a parity wait is only meaningful within one phase).
             const int n0 = group_tiles(n, 0), n1 = group_tiles(n, 1);
             const int nmine = w ? n1 : n0, nother = w ? n0 : n1;
-            ok = (nmine == 0 || ptx::mbar_wait(&B.o_done[w], (cu[w] + nmine - 1) & 1, abort_flag, tmo)) &&
-                 (nother == 0 || ptx::mbar_wait(&B.o_done[w ^ 1], (cu[w ^ 1] + nother - 1) & 1, abort_flag, tmo));
+            ok = (nmine == 0 || ptx::mbar_wait(&B.o_done[w], od[w] & 1, abort_flag, tmo)) &&
+                 (nother == 0 || ptx::mbar_wait(&B.o_done[w ^ 1], od[w ^ 1] & 1, abort_flag, tmo));
+            od[0] += n0 > 0;
+            od[1] += n1 > 0;
             cu[0] += n0;
             cu[1] += n1;
+            t += n;
             if (!ok) break;
             // merge the two groups: exchange (max, sum) per row through shared memory
             float l0, l1;

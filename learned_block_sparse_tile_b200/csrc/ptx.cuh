@@ -62,16 +62,29 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps (without issuing) until
+// the phase completes or about `hint_ns` elapse.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
 // Waits until the phase of parity `parity` of `bar` has completed. Gives up (returns false) when
-// `*abort` becomes non-zero or after `timeout_ns`; on a timeout it raises `*abort` itself.
+// `*abort` becomes non-zero or after `timeout_ns`; on a timeout it raises `*abort` itself. Waiting threads
+// sleep in 100-microsecond slices instead of spinning, so they leave the issue slots to working warps.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > timeout_ns) {
             *abort = 1;

@@ -381,5 +381,6 @@ extern "C" int veda_sync_status(void* stream) {
     if (bits & kErrTimeout) return fail(VEDA_ERR_TIMEOUT, "a bounded device wait expired; the kernel stopped early");
     if (bits & kErrBadList) return fail(VEDA_ERR_BAD_LIST, "a kept list was out of range or not ascending");
     if (bits & kErrBadHead) return fail(VEDA_ERR_INVALID, "a head index was outside [0, H_total)");
+    if (bits & kErrLayout) return fail(VEDA_ERR_CUDA, "attend kernel: shared memory base was not 1024-byte aligned");
     return VEDA_OK;
 }

@@ -154,6 +154,19 @@ int veda_score(const veda_layout* layout, const float* feats_q, const float* fea
                int32_t dim, const float* proj_q, const float* proj_k, void* workspace,
                size_t workspace_bytes, float* scores, void* stream);
 
+/* veda_score without a workspace argument, for callers that cannot allocate device memory when they
+ * need the scores (inside captured graph segments, under a memory pool someone else owns, in loops where
+ * an allocation is not allowed). The pages have no counterpart: this is a service of this library.
+ * Same inputs, outputs and arithmetic as veda_score; the projected features live in one 4 MiB array of
+ * this library's device memory (1,048,576 floats, held by every GPU that loads the library until exit)
+ * and heads are processed in chunks that fit it. Nothing is allocated and nothing needs to start at zero.
+ * The first call on a device looks up the array's device address (make it before any stream capture).
+ * All calls on a device share the array: calls whose kernels overlap on the GPU race and must be
+ * serialised. Errors: VEDA_ERR_UNSUPPORTED when one head needs more than the array holds
+ * (2 * n_video * D > 1,048,576, i.e. n_video > 4096 at D = 128); otherwise as veda_score. */
+int veda_score_noalloc(const veda_layout* layout, const float* feats_q, const float* feats_k, int32_t n_heads,
+                       int32_t dim, const float* proj_q, const float* proj_k, float* scores, void* stream);
+
 /* Head-aware top-k (veda_core.py, "selection", select, block_mask and tile_index_list).
  * Per head and video query row, per column block: empty key tiles are never kept; the row's own tile
  * is kept first when it lies in the block; the other columns are ranked by (score descending, column

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libveda.so"
 
 EXPORTS = [
     "veda_plan", "veda_layout_info", "veda_layout_export", "veda_layout_destroy", "veda_least_padding_box",
-    "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_select", "veda_attend",
+    "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_score_noalloc", "veda_select", "veda_attend",
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
 ]
 
@@ -76,6 +76,7 @@ def lib():
         L.veda_score_workspace_bytes.argtypes = [vp, i32, i32]
         L.veda_score_workspace_bytes.restype = C.c_size_t
         L.veda_score.argtypes = [vp, p, p, i32, i32, p, p, p, C.c_size_t, p, vp]
+        L.veda_score_noalloc.argtypes = [vp, p, p, i32, i32, p, p, p, vp]
         L.veda_select.argtypes = [vp, p, i32, p, p, vp]
         L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_sync_status.argtypes = [vp]
@@ -179,6 +180,13 @@ def veda_score(layout, feats_q, feats_k, proj_q, proj_k, workspace, scores, stre
     _check(lib().veda_score(layout.handle, _ptr(feats_q), _ptr(feats_k), n_heads, dim, _ptr(proj_q), _ptr(proj_k),
                             _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(scores),
                             _stream(stream)))
+
+
+def veda_score_noalloc(layout, feats_q, feats_k, proj_q, proj_k, scores, stream=None):
+    """veda_score without a workspace (for callers that cannot allocate): scratch is the library's own."""
+    n_heads, dim = proj_q.shape[0], proj_q.shape[2]
+    _check(lib().veda_score_noalloc(layout.handle, _ptr(feats_q), _ptr(feats_k), n_heads, dim, _ptr(proj_q),
+                                    _ptr(proj_k), _ptr(scores), _stream(stream)))
 
 
 def veda_select(layout, scores, kept_idx, kept_cnt, stream=None):

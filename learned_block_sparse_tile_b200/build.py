@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libveda.so")
 
-SOURCES = ["veda_api.cu", "veda_plan.cpp"]
+SOURCES = ["veda_api.cu", "veda_plan.cpp", "veda_score_noalloc.cu"]
 HEADERS = ["veda_internal.h", "ptx.cuh", "gather.cuh", "score.cuh", "select.cuh", "attend.cuh"]
 
 

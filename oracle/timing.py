@@ -70,21 +70,26 @@ def _inputs(wl):
 
 
 def time_layer(wl, budget_s=20.0):
-    """One bounded oracle sample (about ``budget_s`` seconds of CPU work), extrapolated to ms/layer."""
+    """One bounded oracle sample (about ``budget_s`` seconds of CPU work), extrapolated to ms/layer.
+
+    The sample grows (more heads per head group, more query tiles) until the CPU work spent on the last
+    sample reaches about half the budget; the estimate of the largest sample is reported."""
     q, k, v, pq, pk = _inputs(wl)
-    heads_sampled = 1
-    items = 16
-    ms, spent, hs, pairs = _sample_layer(wl, q, k, v, pq, pk, heads_sampled, items, seed=0)
-    extra = budget_s - spent
-    if extra > 0 and spent > 0:
-        grow = min(8.0, 1.0 + extra / spent)
-        ms2, spent2, hs, pairs = _sample_layer(wl, q, k, v, pq, pk, max(1, int(heads_sampled * grow)),
-                                               int(items * grow), seed=1)
-        ms, spent = ms2, spent2
+    heads_sampled, items, seed = 1, 16, 0
+    total = 0.0
+    while True:
+        ms, spent, hs, pairs = _sample_layer(wl, q, k, v, pq, pk, heads_sampled, items, seed=seed)
+        total += spent
+        if spent >= budget_s / 2 or total >= budget_s or heads_sampled >= wl.heads:
+            break
+        grow = max(2.0, min(8.0, (budget_s / 2) / max(spent, 1e-3)))
+        heads_sampled = min(wl.heads, int(round(heads_sampled * grow)))
+        items = int(items * grow)
+        seed += 1
     return {"value": round(ms, 1), "unit": "ms/layer", "cores": _threads(), "kind": "oracle",
             "sample": f"{hs} of {wl.heads} heads through layout/gather/pool/logits/select/mask, exact float64 "
                       f"attention on {pairs} attended tile pairs; extrapolated linearly to the whole layer "
-                      f"({spent:.1f} s of CPU work)"}
+                      f"({spent:.1f} s of CPU work in the reported sample, {total:.1f} s in all)"}
 
 
 def reference_arm(wl, steps, warmup, metric, unit, n_gpus=1):

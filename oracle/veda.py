@@ -28,7 +28,7 @@ __all__ = [
     "least_padding_shape", "span_tiles", "build_layout", "gather", "scatter", "pool", "logits",
     "column_blocks", "allowed_per_row", "select", "block_mask", "tile_index_list", "attend_tiles",
     "attend_dense_mask", "dense_attention", "attention_layer", "work_stats", "quantize_fp8_tiles",
-    "attend_tiles_fp8",
+    "attend_tiles_fp8", "layer_spans",
 ]
 
 

@@ -30,7 +30,7 @@ class Case:
         self.tile_refs = not O.keeps_all(self.wl.reference)
 
     def spans_oracle(self, box):
-        return O.veda.layer_spans(self.wl.ref_spans, (self.wl.target[0], self.wl.target[1], box), self.tile_refs)
+        return O.layer_spans(self.wl.ref_spans, (self.wl.target[0], self.wl.target[1], box), self.tile_refs)
 
     def run_group(self, box, heads, out=None):
         """All device stages for one group; returns a dict of host copies plus the layout."""

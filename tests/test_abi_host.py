@@ -70,7 +70,7 @@ def test_plan_matches_oracle_on_workloads(name):
     lps = O.least_padding_shape(wl.target[1])
     tile_refs = not O.keeps_all(wl.reference)
     for shape, _heads in V.head_groups(wl, lambda _: lps):
-        spans = O.veda.layer_spans(wl.ref_spans, (wl.target[0], wl.target[1], shape), tile_refs)
+        spans = O.layer_spans(wl.ref_spans, (wl.target[0], wl.target[1], shape), tile_refs)
         _check_plan(spans, wl.seq_len, wl.generated, wl.reference)
 
 

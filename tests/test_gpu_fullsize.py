@@ -1,0 +1,101 @@
+"""Full-size GPU parity on the published configurations, in the launch configuration bench.py times
+(VedaLayer on the whole layer). Plans and kept lists are compared in full (bit-exact); scores in full
+(relative tolerance); pooled features and attention outputs on seeded samples of query tiles that always
+include the first and last video tiles and the first and last global tiles."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import veda_synth as V
+from learned_block_sparse_tile_b200 import VedaLayer
+from learned_block_sparse_tile_b200 import _lib as L
+from learned_block_sparse_tile_b200 import build as B
+
+from gpu_util import ATT_MAX_ABS, ATT_MEAN_ABS, POOL_ABS, POOL_REL, SCORE_REL, f32
+
+pytestmark = pytest.mark.gpu
+
+_inputs = {}
+
+
+def inputs(wl):
+    """Q/K/V/projections, shared by workloads with the same shapes and seeds (the budget sweep)."""
+    key = (wl.seq_len, wl.heads, wl.dim, wl.ref_spans, wl.target, wl.bias)
+    if key not in _inputs:
+        _inputs.clear()
+        q, k, v = V.make_qkv(wl)
+        pq, pk = V.make_projections(wl)
+        _inputs[key] = dict(q=q, k=k, v=v, pq=pq, pk=pk, dq=q.cuda(), dk=k.cuda(), dv=v.cuda(),
+                            nq=f32(q), nk=f32(k), nv=f32(v))
+    return _inputs[key]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+    L.veda_device_check()
+    yield
+    _inputs.clear()
+
+
+@pytest.mark.parametrize("name", ["single", "mixed", "long", "sweep_tiles24", "sweep_r025", "sweep_r050",
+                                  "sweep_dense"])
+def test_full_size_layer(name):
+    wl = V.workload(name)
+    x = inputs(wl)
+    layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
+                      wl.heads, wl.dim)
+    layer.set_projections(x["pq"], x["pk"])
+    out = torch.full_like(x["dq"], 7.0)
+    layer.forward(x["dq"], x["dk"], x["dv"], out)
+    assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+    got_out = f32(out)
+    tile_refs = not O.keeps_all(wl.reference)
+    rng = np.random.default_rng(7)
+    for g in layer.groups:
+        heads = g["heads_list"]
+        lay_o = O.build_layout(O.layer_spans(wl.ref_spans, (wl.target[0], wl.target[1], g["box"]), tile_refs),
+                               wl.seq_len)
+        perm, vc, _ = L.veda_layout_export(g["layout"])
+        assert np.array_equal(perm, lay_o.perm) and np.array_equal(vc, lay_o.valid_count)
+        # pooled features on sampled tiles
+        sample = V.sample_tiles(lay_o.n_video, lay_o.n_video, 24)
+        D = wl.dim
+        for key, xt in (("feats_q", x["nq"]), ("feats_k", x["nk"])):
+            got = f32(g[key])
+            for i in sample:
+                rows = lay_o.perm[i * 128:(i + 1) * 128]
+                rows = rows[rows >= 0]
+                blk = xt[rows][:, heads, :].astype(np.float64)  # [c, H', D]
+                want = np.concatenate([blk.mean(0), blk.max(0), blk.min(0)], axis=-1)
+                assert np.array_equal(got[:, i, D:], want[:, D:])
+                assert np.all(np.abs(got[:, i, :D] - want[:, :D]) <= POOL_ABS + POOL_REL * np.abs(want[:, :D]))
+        # scores in full, from the GPU's features
+        fq, fk = f32(g["feats_q"]), f32(g["feats_k"])
+        want_s = O.logits(fq, fk, f32(x["pq"][heads]), f32(x["pk"][heads]))
+        got_s = f32(g["scores"])
+        for h in range(len(heads)):
+            assert np.abs(got_s[h] - want_s[h]).max() <= SCORE_REL * np.abs(want_s[h]).max()
+        # kept lists in full, bit-exact on identical scores
+        kept = O.select(got_s, lay_o, O.column_blocks(lay_o, wl.generated, wl.reference))
+        mask = O.block_mask(kept, lay_o)
+        idx, cnt = g["kept_idx"].cpu().numpy(), g["kept_cnt"].cpu().numpy()
+        want_cnt = mask[:, :lay_o.n_video].sum(-1)
+        assert np.array_equal(cnt, want_cnt)
+        for h in range(len(heads)):
+            for r in range(lay_o.n_video):
+                assert np.array_equal(idx[h, r, :cnt[h, r]], np.flatnonzero(mask[h, r])), (h, r)
+        # attention on sampled query tiles of every head
+        q_tiles = V.sample_tiles(lay_o.n_tiles, lay_o.n_video, 3, seed=int(rng.integers(1 << 30)))
+        qt, kt, vt = (O.gather(a, lay_o, heads) for a in (x["nq"], x["nk"], x["nv"]))
+        o_t = O.attend_tiles(qt, kt, vt, lay_o, lambda hh, i: np.flatnonzero(mask[hh, i]), q_tiles=q_tiles)
+        errs = []
+        for i in q_tiles:
+            rows = lay_o.perm[i * 128:(i + 1) * 128]
+            real = rows >= 0
+            for j, hh in enumerate(heads):
+                d = np.abs(got_out[rows[real], hh, :] - o_t[i * 128:(i + 1) * 128][real, j, :])
+                errs.append(d)
+        err = np.concatenate([e.ravel() for e in errs])
+        assert err.max() <= ATT_MAX_ABS and err.mean() <= ATT_MEAN_ABS, (err.max(), err.mean())

@@ -210,6 +210,12 @@ int veda_device_check(void);
 /* Upper bound, in nanoseconds, of every bounded device-side wait (default 1e9). Process-wide. */
 void veda_set_wait_timeout_ns(uint64_t ns);
 
+/* Test hook for the failure path (the pages have no counterpart): the calling thread's next veda_attend
+ * withholds its Q tile loads, so the kernel's waits on them expire; the kernel then lets its in-flight
+ * copies and MMAs finish, frees its tensor memory and returns, and veda_sync_status reports
+ * VEDA_ERR_TIMEOUT. The output of that call is unspecified; the device stays usable. */
+void veda_debug_hold_next_attend(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,6 +21,7 @@ EXPORTS = [
     "veda_plan", "veda_layout_info", "veda_layout_export", "veda_layout_destroy", "veda_least_padding_box",
     "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_score_noalloc", "veda_select", "veda_attend",
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
+    "veda_debug_hold_next_attend",
 ]
 
 
@@ -83,6 +84,8 @@ def lib():
         L.veda_last_error.restype = C.c_char_p
         L.veda_set_wait_timeout_ns.argtypes = [C.c_uint64]
         L.veda_set_wait_timeout_ns.restype = None
+        L.veda_debug_hold_next_attend.argtypes = []
+        L.veda_debug_hold_next_attend.restype = None
         _lib = L
     return _lib
 
@@ -216,3 +219,8 @@ def veda_device_check():
 
 def veda_set_wait_timeout_ns(ns):
     lib().veda_set_wait_timeout_ns(int(ns))
+
+
+def veda_debug_hold_next_attend():
+    """Test hook: the calling thread's next veda_attend withholds its Q loads (its waits expire)."""
+    lib().veda_debug_hold_next_attend()

@@ -44,6 +44,10 @@ constexpr int kErrTimeout = 1;
 constexpr int kErrBadList = 2;
 constexpr int kErrLayout = 8;  // shared memory base not 1024-byte aligned: the kernel did nothing
 
+// Upper bound of the waits that let in-flight copies and MMAs finish before a CTA that gave up exits;
+// independent of the (possibly short) wait limit, since those operations complete in microseconds.
+constexpr uint64_t kDrainNs = 200000000ull;
+
 struct AttendArgs {
     const int32_t* kept_idx;     // [n_heads, n_video, max_kept]
     const int32_t* kept_cnt;     // [n_heads, n_video]
@@ -59,6 +63,7 @@ struct AttendArgs {
     float scale_log2;  // D^-0.5 * log2(e)
     uint64_t timeout_ns;
     int* err;
+    int hold_q;  // test hook: the producer withholds every Q load, so every wait on Q expires
 };
 
 template <int D>
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(384, 1)
             if (kq && bad && lane == 0) atomicOr(a.err, kErrBadList);
             if (n == 0) continue;
             const int32_t row0 = int32_t(int64_t(hh) * a.n_slots);
-            if (kq && lane == 0 && ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo)) {
+            if (kq && lane == 0 && !a.hold_q && ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo)) {
                 ptx::mbar_arrive_expect_tx(&B.q_full, C::kTileBytes);
                 for (int x = 0; x < C::kBoxes; ++x)
                     ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * 64, row0 + qt * 128, &B.q_full);
@@ -246,8 +251,8 @@ __global__ void __launch_bounds__(384, 1)
             // every copy already issued must land before the CTA releases its shared memory
             volatile int never = 0;
             for (int k = (issued > S ? issued - S : 0); k < issued; ++k)
-                ptx::mbar_wait(kq ? &B.k_full[k % KS] : &B.v_full[k % VS], (k / S) & 1, &never, tmo);
-            if (kq && issued_q > 0) ptx::mbar_wait(&B.q_full, (issued_q - 1) & 1, &never, tmo);
+                ptx::mbar_wait(kq ? &B.k_full[k % KS] : &B.v_full[k % VS], (k / S) & 1, &never, kDrainNs);
+            if (kq && issued_q > 0) ptx::mbar_wait(&B.q_full, (issued_q - 1) & 1, &never, kDrainNs);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer (one thread)
@@ -312,7 +317,7 @@ __global__ void __launch_bounds__(384, 1)
             // every MMA issued so far must finish before the TMEM is released
             volatile int never = 0;
             ptx::mma_commit(&B.drain);
-            ptx::mbar_wait(&B.drain, 0, &never, tmo);
+            ptx::mbar_wait(&B.drain, 0, &never, kDrainNs);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------- softmax groups (warps 4-7, 8-11)

@@ -26,6 +26,7 @@ __device__ int g_err;  // latched kernel error bits (kErrTimeout | kErrBadList |
 namespace {
 
 thread_local std::string t_error;
+thread_local bool t_hold_next_attend = false;
 std::atomic<uint64_t> g_timeout_ns{1000000000ull};
 
 struct DeviceState {
@@ -150,6 +151,8 @@ using namespace veda;
 extern "C" const char* veda_last_error(void) { return t_error.c_str(); }
 
 extern "C" void veda_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : 1; }
+
+extern "C" void veda_debug_hold_next_attend(void) { t_hold_next_attend = true; }
 
 extern "C" int veda_device_check(void) {
     clear_error();
@@ -362,6 +365,8 @@ extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const voi
     a.scale_log2 = float((1.0 / std::sqrt(double(dim))) * 1.4426950408889634);
     a.timeout_ns = g_timeout_ns.load();
     a.err = ds->err;
+    a.hold_q = t_hold_next_attend ? 1 : 0;
+    t_hold_next_attend = false;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return dim == 128 ? launch_attend<128>(ds, mq, mk, mv, a, s) : launch_attend<64>(ds, mq, mk, mv, a, s);
 }

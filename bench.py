@@ -115,6 +115,16 @@ class Clocks:
                 "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
 
 
+def max_over_ranks(value, world, device):
+    """The largest of every rank's ``value`` (a time), as a float; collective only over the timings."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def flops_per_pair(dim):
     return 4.0 * 128 * 128 * dim
 
@@ -184,11 +194,7 @@ def run_veda(args, rank, world, local):
     ms_total = t0.elapsed_time(t1)
     stage_ms = {name: sum(a.elapsed_time(b) for a, b in evs) / args.steps for name, evs in stage_ev.items()}
     attend_launch_ms = stage_ms["attend"] / len(layer.groups)
-    ms_step = ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step], device=f"cuda:{local}")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(ms_total / args.steps, world, f"cuda:{local}")
 
     # end to end through the public API: pinned host inputs in, result out, every step
     hq, hk, hv = (x.pin_memory() for x in (q, k, v))
@@ -205,11 +211,7 @@ def run_veda(args, rank, world, local):
         hout.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=f"cuda:{local}")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, f"cuda:{local}")
 
     work = layer.work_tiles()
     pairs = layer.attended_tile_pairs()

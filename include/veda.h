@@ -197,6 +197,26 @@ int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, con
                 void* out, const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
                 void* stream);
 
+/* FP8 Q/K variant, step 1 (not on the pages: their kernel quantises to INT8 by a recipe they do not
+ * print; this follows the FP8 e4m3 variant of the 104k budget sweep). Per (head, 128-row tile) of a
+ * tile-ordered bf16 tensor: scale = amax(|x|) over the tile's real rows / 448 (1 when 0), and each code is
+ * x / scale rounded to nearest-even e4m3 with saturation at +-448 (padding rows stay 0).
+ *  x_t     device bf16 [n_heads, N, D] (from veda_gather).
+ *  codes   device e4m3 bytes [n_heads, N, D] out.
+ *  scales  device fp32 [n_heads, n_tiles] out.
+ * D must be 64 or 128. */
+int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim, void* codes,
+                      float* scales, void* stream);
+
+/* FP8 Q/K variant, step 2: veda_attend with Q and K given as e4m3 codes and per-tile scales (from
+ * veda_quantize_fp8); S = Q K^T runs as an e4m3 x e4m3 tensor-core product with fp32 accumulation and is
+ * multiplied by scale_q(query tile) * scale_k(key tile) * D^-0.5; P and V stay bf16. Selection is not
+ * affected (it pools the bf16 Q and K). D must be 128. Other arguments and errors as veda_attend. */
+int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* k_codes, const float* scales_q,
+                    const float* scales_k, const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
+                    const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
+                    const int32_t* heads, void* stream);
+
 /* Synchronizes `stream`, then reads and clears this device's latched kernel error word.
  * Returns VEDA_OK, VEDA_ERR_TIMEOUT, VEDA_ERR_BAD_LIST or VEDA_ERR_CUDA. */
 int veda_sync_status(void* stream);

@@ -21,7 +21,7 @@ EXPORTS = [
     "veda_plan", "veda_layout_info", "veda_layout_export", "veda_layout_destroy", "veda_least_padding_box",
     "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_score_noalloc", "veda_select", "veda_attend",
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
-    "veda_debug_hold_next_attend",
+    "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_attend_fp8",
 ]
 
 
@@ -80,6 +80,8 @@ def lib():
         L.veda_score_noalloc.argtypes = [vp, p, p, i32, i32, p, p, p, vp]
         L.veda_select.argtypes = [vp, p, i32, p, p, vp]
         L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
+        L.veda_quantize_fp8.argtypes = [vp, p, i32, i32, p, p, vp]
+        L.veda_attend_fp8.argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_sync_status.argtypes = [vp]
         L.veda_last_error.restype = C.c_char_p
         L.veda_set_wait_timeout_ns.argtypes = [C.c_uint64]
@@ -202,6 +204,19 @@ def veda_attend(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, stream=No
     _check(lib().veda_attend(layout.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), q_t.shape[0], q_t.shape[2],
                              _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1], _ptr(heads),
                              _stream(stream)))
+
+
+def veda_quantize_fp8(layout, x_t, codes, scales, stream=None):
+    """x_t: bf16 [n, N, D]; codes: uint8 [n, N, D] (e4m3 bytes); scales: fp32 [n, n_tiles]."""
+    _check(lib().veda_quantize_fp8(layout.handle, _ptr(x_t), x_t.shape[0], x_t.shape[2], _ptr(codes), _ptr(scales),
+                                   _stream(stream)))
+
+
+def veda_attend_fp8(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx, kept_cnt, out, heads, stream=None):
+    """veda_attend with e4m3 Q/K codes (uint8 [n, N, D]) and their per-tile scales."""
+    _check(lib().veda_attend_fp8(layout.handle, _ptr(q_codes), _ptr(k_codes), _ptr(scales_q), _ptr(scales_k),
+                                 _ptr(v_t), v_t.shape[0], v_t.shape[2], _ptr(kept_idx), _ptr(kept_cnt), _ptr(out),
+                                 _strides(out), out.shape[1], _ptr(heads), _stream(stream)))
 
 
 def veda_sync_status(stream=None):

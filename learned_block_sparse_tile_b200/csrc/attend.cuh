@@ -64,34 +64,40 @@ struct AttendArgs {
     uint64_t timeout_ns;
     int* err;
     int hold_q;  // test hook: the producer withholds every Q load, so every wait on Q expires
+    const float* scales_q;  // FP8 variant: [n_heads, n_tiles] per-tile scales of the e4m3 Q and K codes
+    const float* scales_k;
 };
 
-template <int D>
+// kFp8: Q and K are e4m3 codes with per-tile scales (S = Q K^T on the kind::f8f6f4 path); V stays bf16.
+template <int D, bool kFp8 = false>
 struct AttendCfg {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(!kFp8 || D == 128, "the FP8 Q/K variant is built for head_dim 128");
     static constexpr int kWarps = 12;
     static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kTileBytes = 128 * D * 2;  // one Q, K or V tile (bf16)
-    static constexpr int kBoxes = D / 64;           // 64-column TMA boxes per tile
-    static constexpr int kKStages = 3;              // K ring depth
-    static constexpr int kVStages = 3;              // V ring depth
+    static constexpr int kQKBytes = 128 * D * (kFp8 ? 1 : 2);  // one Q or K tile
+    static constexpr int kTileBytes = 128 * D * 2;             // one V tile (bf16)
+    static constexpr int kBoxesQK = kFp8 ? 1 : D / 64;         // 128-byte-wide TMA boxes per Q/K tile
+    static constexpr int kBoxes = D / 64;                      // 64-column (128-byte) TMA boxes per V tile
+    static constexpr int kKStages = kFp8 ? 4 : 3;              // K ring depth
+    static constexpr int kVStages = kFp8 ? 4 : 3;              // V ring depth
     // header (barriers, then the [2 groups][128 rows] (max, sum) exchange) first, then the 1024-aligned
     // tiles; with a 1024-aligned dynamic base this fills the 227 KB a CTA may use at head_dim 128
     static constexpr int kOffBar = 0;
     static constexpr int kOffStats = 256;
     static constexpr int kHeader = 3072;
     static constexpr int kOffQ = kHeader;
-    static constexpr int kOffK = kOffQ + kTileBytes;
-    static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+    static constexpr int kOffK = kOffQ + kQKBytes;
+    static constexpr int kOffV = kOffK + kKStages * kQKBytes;
     static constexpr int kSmem = kOffV + kVStages * kTileBytes;
     static constexpr uint32_t kTmemCols = 512;  // S/P of group 0, S/P of group 1, O of group 0, O of group 1
-    static constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
+    static constexpr uint32_t kIdescS = kFp8 ? ptx::idesc_e4m3_f32(128, 128) : ptx::idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, false, true);
 };
 
 struct AttendBars {
     uint64_t q_full, q_empty;
-    uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+    uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2], o_done[2];
     uint64_t o_empty, merge, drain;
 };
@@ -152,11 +158,11 @@ __device__ __forceinline__ void decode_item(const AttendArgs& a, int item, int* 
 // Tiles of an item that softmax group w handles: the item-local tiles j = w, w + 2, ...
 __device__ __forceinline__ int group_tiles(int n, int w) { return (n - w + 1) >> 1; }
 
-template <int D>
+template <int D, bool kFp8>
 __global__ void __launch_bounds__(384, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const AttendArgs a) {
-    using C = AttendCfg<D>;
+    using C = AttendCfg<D, kFp8>;
     constexpr int KS = C::kKStages, VS = C::kVStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw;
@@ -219,9 +225,9 @@ __global__ void __launch_bounds__(384, 1)
             if (n == 0) continue;
             const int32_t row0 = int32_t(int64_t(hh) * a.n_slots);
             if (kq && lane == 0 && !a.hold_q && ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo)) {
-                ptx::mbar_arrive_expect_tx(&B.q_full, C::kTileBytes);
-                for (int x = 0; x < C::kBoxes; ++x)
-                    ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * 64, row0 + qt * 128, &B.q_full);
+                ptx::mbar_arrive_expect_tx(&B.q_full, C::kQKBytes);
+                for (int x = 0; x < C::kBoxesQK; ++x)
+                    ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * (kFp8 ? 128 : 64), row0 + qt * 128, &B.q_full);
                 ++issued_q;
             }
             __syncwarp();
@@ -234,11 +240,13 @@ __global__ void __launch_bounds__(384, 1)
                     const int st = issued % S, u = issued / S;
                     uint64_t* empty = kq ? &B.k_empty[st] : &B.v_empty[st];
                     uint64_t* full = kq ? &B.k_full[st] : &B.v_full[st];
-                    uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * C::kTileBytes;
+                    const int bytes = kq ? C::kQKBytes : C::kTileBytes;
+                    uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * bytes;
                     if (ptx::mbar_wait(empty, (u & 1) ^ 1, abort_flag, tmo)) {
-                        ptx::mbar_arrive_expect_tx(full, C::kTileBytes);
-                        for (int x = 0; x < C::kBoxes; ++x)
-                            ptx::tma_load_2d_hint(dst + x * 16384, kq ? &tm_k : &tm_v, x * 64, y, full, keep);
+                        ptx::mbar_arrive_expect_tx(full, bytes);
+                        const int boxes = kq ? C::kBoxesQK : C::kBoxes, xstep = (kq && kFp8) ? 128 : 64;
+                        for (int x = 0; x < boxes; ++x)
+                            ptx::tma_load_2d_hint(dst + x * 16384, kq ? &tm_k : &tm_v, x * xstep, y, full, keep);
                         ++issued;
                     }
                 }
@@ -294,12 +302,20 @@ __global__ void __launch_bounds__(384, 1)
                         ok = ptx::mbar_wait(&B.k_full[st], (tk / KS) & 1, abort_flag, tmo);
                         if (!ok) break;
                         ptx::tc_fence_after();
-                        const uint32_t k0 = ptx::smem_addr(smem + C::kOffK + st * C::kTileBytes);
+                        const uint32_t k0 = ptx::smem_addr(smem + C::kOffK + st * C::kQKBytes);
+                        if constexpr (kFp8) {
+                            // e4m3: a 128-byte row holds all 128 dims; K = 32 per MMA
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                            ptx::mma_bf16_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
-                                             ptx::smem_desc_sw128(k0 + off, 16, 1024), C::kIdescS, kk > 0);
+                            for (int kk = 0; kk < 4; ++kk)
+                                ptx::mma_f8_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + kk * 32, 16, 1024),
+                                               ptx::smem_desc_sw128(k0 + kk * 32, 16, 1024), C::kIdescS, kk > 0);
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                                ptx::mma_bf16_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
+                                                 ptx::smem_desc_sw128(k0 + off, 16, 1024), C::kIdescS, kk > 0);
+                            }
                         }
                         ptx::mma_commit(&B.s_full[w]);  // the softmax group also frees the K slot on it
                         if (j == n - 1) ptx::mma_commit(&B.q_empty);
@@ -328,8 +344,6 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t t_s = tmem + lane_base + 128 * w;        // S / P of this group
         const uint32_t t_o = tmem + lane_base + 256 + 128 * w;  // O of this group
         const uint32_t t_o0 = tmem + lane_base + 256;
-        const float sl2 = a.scale_log2;
-        const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
         int cu[2] = {0, 0};  // tiles each group has had so far (barrier phases)
         int it = 0, t = 0;   // items with tiles so far; tiles so far (K ring positions)
         int od[2] = {0, 0};  // o_done phases: one per item in which the group had a tile
@@ -360,12 +374,19 @@ __global__ void __launch_bounds__(384, 1)
             uint64_t lsum = ptx::f2_pack(0.f, 0.f);
             bool ok = true;
             int my_vc = 128;
+            float my_sk = 1.f;
+            const float sq = kFp8 ? __ldg(a.scales_q + int64_t(hh) * a.n_tiles + qt) : 1.f;
             for (int k = 0; k < nw; ++k) {
                 if ((k & 31) == 0) {
                     const int jj = 2 * (k + lane) + w;
-                    my_vc = jj < n ? __ldg(a.valid_count + __ldg(list + jj)) : 128;
+                    const int tile = jj < n ? __ldg(list + jj) : -1;
+                    my_vc = tile >= 0 ? __ldg(a.valid_count + tile) : 128;
+                    if (kFp8) my_sk = tile >= 0 ? __ldg(a.scales_k + int64_t(hh) * a.n_tiles + tile) : 1.f;
                 }
                 const int vc = __shfl_sync(0xffffffffu, my_vc, k & 31);
+                // log2-domain scale of this tile's logits (the FP8 path also undoes both tiles' scales)
+                const float sl2 = kFp8 ? a.scale_log2 * (sq * __shfl_sync(0xffffffffu, my_sk, k & 31)) : a.scale_log2;
+                const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
                 const int idx = cu[w] + k;
                 ok = ptx::mbar_wait(&B.s_full[w], idx & 1, abort_flag, tmo);
                 if (!ok) break;

@@ -16,6 +16,7 @@
 #include "score.cuh"
 #include "select.cuh"
 #include "attend.cuh"
+#include "quant.cuh"
 
 namespace veda {
 
@@ -33,7 +34,7 @@ struct DeviceState {
     bool init = false;
     int sms = 0;
     int* err = nullptr;  // device address of g_err
-    bool attend_attr[2] = {false, false};
+    bool attend_attr[4] = {false, false, false, false};
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -119,16 +120,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2D map over a head-major tile-ordered bf16 tensor viewed as [rows, D]: boxes of 128 rows x 64 columns
-// (128 bytes) with the 128-byte swizzle the MMA descriptors expect.
-int make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int dim) {
+// 2D map over a head-major tile-ordered tensor viewed as [rows, D]: boxes of 128 rows x 128 bytes (64 bf16
+// or 128 e4m3 columns) with the 128-byte swizzle the MMA descriptors expect.
+int make_tile_map(CUtensorMap* m, const void* base, int64_t rows, int dim, bool fp8 = false) {
     auto enc = tensor_map_encoder();
     if (!enc) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int esize = fp8 ? 1 : 2;
     cuuint64_t gdim[2] = {cuuint64_t(dim), cuuint64_t(rows)};
-    cuuint64_t gstride[1] = {cuuint64_t(dim) * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint64_t gstride[1] = {cuuint64_t(dim) * esize};
+    cuuint32_t box[2] = {cuuint32_t(128 / esize), 128};
     cuuint32_t estride[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+    CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void*>(base), gdim, gstride, box, estride,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
@@ -306,42 +309,45 @@ extern "C" int veda_select(const veda_layout* layout, const float* scores, int32
     return launch_check("select_kernel");
 }
 
-template <int D>
+template <int D, bool kFp8>
 static int launch_attend(DeviceState* ds, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttendArgs& a, cudaStream_t s) {
-    using C = AttendCfg<D>;
-    if (!ds->attend_attr[D == 128]) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    using C = AttendCfg<D, kFp8>;
+    const int slot = (D == 128) + 2 * kFp8;
+    if (!ds->attend_attr[slot]) {
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
-        ds->attend_attr[D == 128] = true;
+        ds->attend_attr[slot] = true;
     }
     const int grid = std::max(1, std::min(a.n_items, ds->sms));
-    attend_kernel<D><<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, a);
+    attend_kernel<D, kFp8><<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, a);
     return launch_check("attend_kernel");
 }
 
-extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
-                           int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
-                           const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
-    clear_error();
-    if (!layout || !q_t || !k_t || !v_t || !kept_idx || !kept_cnt || !out || !heads)
-        return fail(VEDA_ERR_INVALID, "veda_attend: NULL argument");
-    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_attend: head_dim must be 64 or 128");
-    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_attend: head counts must be positive");
-    if (int rc = check_strided(out_strides, out, "veda_attend out")) return rc;
-    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t))
-        return fail(VEDA_ERR_INVALID, "veda_attend: tile-ordered inputs need 16-byte alignment");
+static int attend_common(const veda_layout* layout, const void* q, const void* k, const float* sq, const float* sk,
+                         const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
+                         const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
+                         const int32_t* heads, void* stream, bool fp8) {
+    const char* who = fp8 ? "veda_attend_fp8" : "veda_attend";
+    if (!layout || !q || !k || !v_t || !kept_idx || !kept_cnt || !out || !heads || (fp8 && (!sq || !sk)))
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
+    if (fp8 ? dim != 128 : (dim != 64 && dim != 128))
+        return fail(VEDA_ERR_INVALID, std::string(who) + (fp8 ? ": head_dim must be 128" : ": head_dim must be 64 or 128"));
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, std::string(who) + ": head counts must be positive");
+    if (int rc = check_strided(out_strides, out, who)) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v_t))
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": tile-ordered inputs need 16-byte alignment");
     const veda_layout_desc& d = layout->desc;
     if (int64_t(n_heads) * d.n_slots >= (int64_t(1) << 31))
-        return fail(VEDA_ERR_UNSUPPORTED, "veda_attend: n_heads * N must stay below 2^31 rows");
+        return fail(VEDA_ERR_UNSUPPORTED, std::string(who) + ": n_heads * N must stay below 2^31 rows");
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
     const DeviceCopy* dc;
     if (int rc = device_copy(layout, &dc)) return rc;
     CUtensorMap mq, mk, mv;
     const int64_t rows = int64_t(n_heads) * d.n_slots;
-    if (int rc = make_tile_map(&mq, q_t, rows, dim)) return rc;
-    if (int rc = make_tile_map(&mk, k_t, rows, dim)) return rc;
+    if (int rc = make_tile_map(&mq, q, rows, dim, fp8)) return rc;
+    if (int rc = make_tile_map(&mk, k, rows, dim, fp8)) return rc;
     if (int rc = make_tile_map(&mv, v_t, rows, dim)) return rc;
     AttendArgs a;
     a.kept_idx = kept_idx;
@@ -367,8 +373,56 @@ extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const voi
     a.err = ds->err;
     a.hold_q = t_hold_next_attend ? 1 : 0;
     t_hold_next_attend = false;
+    a.scales_q = sq;
+    a.scales_k = sk;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return dim == 128 ? launch_attend<128>(ds, mq, mk, mv, a, s) : launch_attend<64>(ds, mq, mk, mv, a, s);
+    if (fp8) return launch_attend<128, true>(ds, mq, mk, mv, a, s);
+    return dim == 128 ? launch_attend<128, false>(ds, mq, mk, mv, a, s) : launch_attend<64, false>(ds, mq, mk, mv, a, s);
+}
+
+extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
+                           int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                           const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
+    clear_error();
+    return attend_common(layout, q_t, k_t, nullptr, nullptr, v_t, n_heads, dim, kept_idx, kept_cnt, out, out_strides,
+                         h_total, heads, stream, false);
+}
+
+extern "C" int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* k_codes,
+                               const float* scales_q, const float* scales_k, const void* v_t, int32_t n_heads,
+                               int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                               const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
+    clear_error();
+    return attend_common(layout, q_codes, k_codes, scales_q, scales_k, v_t, n_heads, dim, kept_idx, kept_cnt, out,
+                         out_strides, h_total, heads, stream, true);
+}
+
+extern "C" int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim,
+                                 void* codes, float* scales, void* stream) {
+    clear_error();
+    if (!layout || !x_t || !codes || !scales) return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: head_dim must be 64 or 128");
+    if (n_heads <= 0) return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: n_heads must be positive");
+    if (!aligned16(x_t) || !aligned16(codes) || !aligned16(scales))
+        return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: buffers need 16-byte alignment");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    QuantArgs a;
+    a.x_t = static_cast<const __nv_bfloat16*>(x_t);
+    a.valid_count = dc->valid_count;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.n_slots = layout->desc.n_slots;
+    a.n_tiles = layout->desc.n_tiles;
+    dim3 grid(unsigned(layout->desc.n_tiles), unsigned(n_heads));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dim == 128)
+        quantize_fp8_kernel<128><<<grid, 256, 0, s>>>(a);
+    else
+        quantize_fp8_kernel<64><<<grid, 256, 0, s>>>(a);
+    return launch_check("quantize_fp8_kernel");
 }
 
 extern "C" int veda_sync_status(void* stream) {

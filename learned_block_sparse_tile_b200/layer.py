@@ -24,8 +24,9 @@ class VedaLayer:
 
     LAUNCHES_PER_GROUP = 8  # gather q, gather k, 3 score GEMMs, select, gather v, attend
 
-    def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda"):
+    def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False):
         self.seq_len, self.heads, self.dim = int(seq_len), int(heads), int(dim)
+        self.fp8_qk = bool(fp8_qk)
         self.device = torch.device(device)
         lps = L.veda_least_padding_box(target[1])
         groups = {}
@@ -50,8 +51,13 @@ class VedaLayer:
                      scores=torch.empty(n, lay.n_video, lay.n_video, dtype=torch.float32, device=dev),
                      kept_idx=torch.empty(n, lay.n_video, lay.max_kept, dtype=torch.int32, device=dev),
                      kept_cnt=torch.empty(n, lay.n_video, dtype=torch.int32, device=dev))
+            if self.fp8_qk:
+                g.update(q8=torch.empty(n, lay.n_slots, dim, dtype=torch.uint8, device=dev),
+                         k8=torch.empty(n, lay.n_slots, dim, dtype=torch.uint8, device=dev),
+                         sq=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev),
+                         sk=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev))
             self.groups.append(g)
-        self.launches = self.LAUNCHES_PER_GROUP * len(self.groups)
+        self.launches = (self.LAUNCHES_PER_GROUP + 2 * self.fp8_qk) * len(self.groups)
 
     def set_projections(self, proj_q, proj_k):
         """proj_q, proj_k: fp32 [H, 3D, D] (any device); each group keeps its heads' slices on device."""
@@ -86,7 +92,8 @@ class VedaLayer:
         """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten.
 
         ``events``: optional dict; CUDA event pairs recorded around each stage on ``stream`` are appended
-        under the stage names gather_qk, score, select, gather_v and attend (the page's PhaseTimer)."""
+        under the stage names gather_qk, score, select, gather_v, quantize (FP8 Q/K only) and attend (the
+        page's PhaseTimer)."""
         st = stream if stream is not None else torch.cuda.current_stream()
 
         def mark(name):
@@ -118,7 +125,17 @@ class VedaLayer:
             m = mark("gather_v")
             L.veda_gather(lay, v, g["heads"], g["v_t"], None, st)
             done(m)
-            m = mark("attend")
-            L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
-            done(m)
+            if self.fp8_qk:
+                m = mark("quantize")
+                L.veda_quantize_fp8(lay, g["q_t"], g["q8"], g["sq"], st)
+                L.veda_quantize_fp8(lay, g["k_t"], g["k8"], g["sk"], st)
+                done(m)
+                m = mark("attend")
+                L.veda_attend_fp8(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"],
+                                  out, g["heads"], st)
+                done(m)
+            else:
+                m = mark("attend")
+                L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
+                done(m)
         return out

@@ -40,12 +40,12 @@ def built():
 
 
 @pytest.mark.parametrize("name", ["single", "mixed", "long", "sweep_tiles24", "sweep_r025", "sweep_r050",
-                                  "sweep_dense"])
+                                  "sweep_dense", "sweep_fp8"])
 def test_full_size_layer(name):
     wl = V.workload(name)
     x = inputs(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim)
+                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk)
     layer.set_projections(x["pq"], x["pk"])
     out = torch.full_like(x["dq"], 7.0)
     layer.forward(x["dq"], x["dk"], x["dv"], out)
@@ -89,13 +89,31 @@ def test_full_size_layer(name):
         # attention on sampled query tiles of every head
         q_tiles = V.sample_tiles(lay_o.n_tiles, lay_o.n_video, 3, seed=int(rng.integers(1 << 30)))
         qt, kt, vt = (O.gather(a, lay_o, heads) for a in (x["nq"], x["nk"], x["nv"]))
-        o_t = O.attend_tiles(qt, kt, vt, lay_o, lambda hh, i: np.flatnonzero(mask[hh, i]), q_tiles=q_tiles)
-        errs = []
-        for i in q_tiles:
-            rows = lay_o.perm[i * 128:(i + 1) * 128]
-            real = rows >= 0
-            for j, hh in enumerate(heads):
-                d = np.abs(got_out[rows[real], hh, :] - o_t[i * 128:(i + 1) * 128][real, j, :])
-                errs.append(d)
-        err = np.concatenate([e.ravel() for e in errs])
+        lists = lambda hh, i: np.flatnonzero(mask[hh, i])
+        attend = O.attend_tiles_fp8 if wl.fp8_qk else O.attend_tiles
+        o_t = attend(qt, kt, vt, lay_o, lists, q_tiles=q_tiles)
+        err = _sampled_error(got_out, o_t, lay_o, heads, q_tiles)
         assert err.max() <= ATT_MAX_ABS and err.mean() <= ATT_MEAN_ABS, (err.max(), err.mean())
+        if wl.fp8_qk:
+            # against unquantised attention: no worse than the FP8 reading's own quantisation error
+            o_ref = O.attend_tiles(qt, kt, vt, lay_o, lists, q_tiles=q_tiles)
+            q_err = _sampled_error(o_t, o_ref, lay_o, list(range(len(heads))), q_tiles, packed=False)
+            err_ref = _sampled_error(got_out, o_ref, lay_o, heads, q_tiles)
+            assert err_ref.max() <= q_err.max() + ATT_MAX_ABS, (err_ref.max(), q_err.max())
+            assert err_ref.max() <= FP8_REPORT_CAP, err_ref.max()
+
+
+FP8_REPORT_CAP = 1.0  # sanity cap; the e4m3 reading itself moves outputs by a few 1e-1 on this data
+
+
+def _sampled_error(got, want_t, lay_o, heads, q_tiles, packed=True):
+    """|got - want| over the real rows of the sampled query tiles; got is packed [S, H, D] (or tile-ordered
+    [N, H', D] when packed is False), want_t tile-ordered [N, H', D]."""
+    errs = []
+    for i in q_tiles:
+        rows = lay_o.perm[i * 128:(i + 1) * 128]
+        real = rows >= 0
+        for j, hh in enumerate(heads):
+            g = got[rows[real], hh, :] if packed else got[i * 128:(i + 1) * 128][real, j, :]
+            errs.append(np.abs(g - want_t[i * 128:(i + 1) * 128][real, j, :]).ravel())
+    return np.concatenate(errs)

@@ -150,3 +150,44 @@ def test_bad_arguments_rejected_on_host():
     with pytest.raises(L.VedaError):  # workspace too small
         L.veda_score(lay, res["fq"], res["fk"], c.pq[heads].cuda(), c.pk[heads].cuda(),
                      torch.empty(4, device="cuda"), res["scores"])
+
+
+def test_fp8_qk_variant():
+    # quantiser: scales and codes equal to the oracle's reading bit for bit;
+    # attention: against the oracle's FP8 reading (tight) and against unquantised attention (5e-2)
+    c = case("small_d128")
+    wl = c.wl
+    q, k, v = f32(c.q), f32(c.k), f32(c.v)
+    out = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    want_fp8 = np.full(out.shape, np.nan)
+    want_ref = np.full(out.shape, np.nan)
+    for box, heads in c.groups:
+        res = c.run_group(box, heads)
+        lay = res["layout"]
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        n = len(heads)
+        q8 = torch.empty(n, lay.n_slots, wl.dim, dtype=torch.uint8, device="cuda")
+        k8 = torch.empty_like(q8)
+        sq = torch.empty(n, lay.n_tiles, dtype=torch.float32, device="cuda")
+        sk = torch.empty_like(sq)
+        L.veda_quantize_fp8(lay, res["q_t"], q8, sq)
+        L.veda_quantize_fp8(lay, res["k_t"], k8, sk)
+        L.veda_attend_fp8(lay, q8, k8, sq, sk, res["v_t"], res["kept_idx"], res["kept_cnt"], out, res["heads"])
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        qt, kt, vt = (O.gather(x, lay_o, heads) for x in (q, k, v))
+        for x_t, codes, scales in ((qt, q8, sq), (kt, k8, sk)):
+            want_codes, want_scales = O.quantize_fp8_tiles(x_t, lay_o)
+            assert np.array_equal(f32(scales).astype(np.float64), want_scales)
+            got_codes = codes.view(torch.float8_e4m3fn).float().cpu().numpy().transpose(1, 0, 2)
+            assert np.array_equal(got_codes, want_codes)
+        _, mask = oracle_kept(lay_o, f32(res["scores"]), O.column_blocks(lay_o, wl.generated, wl.reference))
+        lists = lambda hh, i: np.flatnonzero(mask[hh, i])
+        O.scatter(want_fp8, O.attend_tiles_fp8(qt, kt, vt, lay_o, lists), lay_o, heads)
+        O.scatter(want_ref, O.attend_tiles(qt, kt, vt, lay_o, lists), lay_o, heads)
+    got = f32(out)
+    mx, mean = attention_error(got, want_fp8)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    # against unquantised attention the kernel adds nothing beyond the reading's own quantisation error
+    mx, _ = attention_error(got, want_ref)
+    q_err, _ = attention_error(want_fp8, want_ref)
+    assert mx <= q_err + ATT_MAX_ABS, (mx, q_err)

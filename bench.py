@@ -132,7 +132,7 @@ def flops_per_pair(dim):
 def stage_bytes(layer, wl):
     """Algorithmic HBM bytes per launch of each stage, summed over head groups."""
     D, S = wl.dim, wl.seq_len
-    out = {"gather_qk": 0, "score": 0, "select": 0, "gather_v": 0, "attend": 0}
+    out = {"gather_qk": 0, "score": 0, "select": 0, "gather_v": 0, "quantize": 0, "attend": 0}
     for g in layer.groups:
         lay, n = g["layout"], len(g["heads_list"])
         real = n * S * D * 2
@@ -147,6 +147,8 @@ def stage_bytes(layer, wl):
         kept = int(g["kept_cnt"].sum())
         out["select"] += sc + 4 * (kept + n * lay.n_video)
         out["attend"] += slots + real + 4 * (kept + n * lay.n_video)  # Q in, O out, lists; K/V counted as L2 reuse
+        if layer.fp8_qk:
+            out["quantize"] += 2 * (slots + slots // 2)  # bf16 Q and K tiles in, e4m3 codes out
     return out
 
 
@@ -160,7 +162,7 @@ def run_veda(args, rank, world, local):
     q, k, v = V.make_qkv(wl)
     pq, pk = V.make_projections(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim, device=f"cuda:{local}")
+                      wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk)
     layer.set_projections(pq, pk)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     out = torch.empty_like(dq)
@@ -229,7 +231,8 @@ def run_veda(args, rank, world, local):
     res = {
         "metric": METRIC, "value": round(ms_step / world, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 Q/K, bf16 P/V" if wl.fp8_qk else "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V with a low-rank locality bias; random predictor projections)",
         "config": {"workload": f"{wl.name}: {wl.note}", "seq_len": wl.seq_len, "heads": wl.heads,
                    "head_dim": wl.dim, "budget": {"generated": wl.generated, "reference": wl.reference},

@@ -12,7 +12,10 @@
 // item. While one group computes its softmax the tensor core works on the other group's tiles.
 //   warp 0       TMA producer of Q (one buffer) and K (ring of 3); warp 2: TMA producer of V (ring of 3).
 //                Every box is 128 rows x 128 bytes with the 128-byte swizzle.
-//   warp 1       TMEM owner and MMA issuer (one thread): S_j = Q K_j^T (both operands in shared memory) into
+//   warp 1       TMEM owner and MMA issuer: the whole warp runs the issue loop (its waits, descriptors and
+//                ring positions are warp-uniform) and elect.sync lets one lane issue each tcgen05 instruction,
+//                which keeps the issuer's instruction count low next to the softmax warps sharing its
+//                sub-partition. S_j = Q K_j^T (both operands in shared memory) into
 //                the S columns of group j%2, then O_(j%2) += P_j V_j with P read from TMEM where the group
 //                left it (the "TS" form) and V from shared memory. Issue order per item: S_0, S_1, then per
 //                tile PV_j followed by S_(j+2).
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(384, 1)
                 ++issued_q;
             }
             __syncwarp();
-            if (*abort_flag) break;
+            if (__any_sync(0xffffffffu, *abort_flag)) break;
             int mine = 0;
             for (int j = 0; j < n; ++j) {
                 if ((j & 31) == 0) mine = (j + lane < n) ? __ldg(list + j + lane) : 0;
@@ -251,9 +254,9 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
                 __syncwarp();
-                if (*abort_flag) break;
+                if (__any_sync(0xffffffffu, *abort_flag)) break;
             }
-            if (*abort_flag) break;
+            if (__any_sync(0xffffffffu, *abort_flag)) break;
         }
         if (*abort_flag && lane == 0) {
             // every copy already issued must land before the CTA releases its shared memory
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(384, 1)
             if (kq && issued_q > 0) ptx::mbar_wait(&B.q_full, (issued_q - 1) & 1, &never, kDrainNs);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------- MMA issuer (one thread)
+        // ------------------------------------------------------------- MMA issuer (whole warp, one lane issues)
         // Per item: S_0 and S_1, then for each tile j: O_(j%2) += P_j V_j, then S_(j+2). S_j lands in S
         // buffer j%2, which softmax group j%2 turns into P_j in place.
         int it = 0, t = 0;      // items with tiles so far; tiles so far (ring positions)
@@ -275,9 +278,9 @@ __global__ void __launch_bounds__(384, 1)
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
             if (n == 0) continue;
-            if (lane == 0) {
+            {
                 const uint32_t q0 = ptx::smem_addr(smem + C::kOffQ);
-                bool ok = ptx::mbar_wait(&B.q_full, it & 1, abort_flag, tmo);
+                bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_full, it & 1, abort_flag, tmo));
                 for (int j = 0; ok && j < n + 2; ++j) {
                     if (j >= 2) {
                         // O_w += P V for tile jj = j - 2
@@ -285,21 +288,22 @@ __global__ void __launch_bounds__(384, 1)
                         ok = ptx::mbar_wait(&B.p_full[w], idx & 1, abort_flag, tmo) &&
                              ptx::mbar_wait(&B.v_full[sv], (tv / VS) & 1, abort_flag, tmo) &&
                              (jj > 0 || ptx::mbar_wait(&B.o_empty, (it & 1) ^ 1, abort_flag, tmo));
+                        ok = __all_sync(0xffffffffu, ok);
                         if (!ok) break;
                         ptx::tc_fence_after();
                         const uint32_t v0 = ptx::smem_addr(smem + C::kOffV + sv * C::kTileBytes);
                         const uint32_t o = tmem + 256 + 128 * w, p = tmem + 128 * w;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            ptx::mma_bf16_ts(o, p + kk * 8, ptx::smem_desc_sw128(v0 + kk * 2048, 16384, 1024), C::kIdescPV,
+                            ptx::mma_bf16_ts_w(o, p + kk * 8, ptx::smem_desc_sw128(v0 + kk * 2048, 16384, 1024), C::kIdescPV,
                                              (jj >= 2 || kk > 0) ? 1u : 0u);
-                        ptx::mma_commit(&B.v_empty[sv]);
-                        if (jj >= n - 2) ptx::mma_commit(&B.o_done[w]);  // the group's last tile of the item
+                        ptx::mma_commit_w(&B.v_empty[sv]);
+                        if (jj >= n - 2) ptx::mma_commit_w(&B.o_done[w]);  // the group's last tile of the item
                     }
                     if (j < n) {
                         // S_j = Q K_j^T into S buffer j%2
                         const int w = j & 1, tk = t + j, st = tk % KS;
-                        ok = ptx::mbar_wait(&B.k_full[st], (tk / KS) & 1, abort_flag, tmo);
+                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.k_full[st], (tk / KS) & 1, abort_flag, tmo));
                         if (!ok) break;
                         ptx::tc_fence_after();
                         const uint32_t k0 = ptx::smem_addr(smem + C::kOffK + st * C::kQKBytes);
@@ -307,18 +311,18 @@ __global__ void __launch_bounds__(384, 1)
                             // e4m3: a 128-byte row holds all 128 dims; K = 32 per MMA
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                ptx::mma_f8_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + kk * 32, 16, 1024),
+                                ptx::mma_f8_ss_w(tmem + 128 * w, ptx::smem_desc_sw128(q0 + kk * 32, 16, 1024),
                                                ptx::smem_desc_sw128(k0 + kk * 32, 16, 1024), C::kIdescS, kk > 0);
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                                ptx::mma_bf16_ss(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
+                                ptx::mma_bf16_ss_w(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
                                                  ptx::smem_desc_sw128(k0 + off, 16, 1024), C::kIdescS, kk > 0);
                             }
                         }
-                        ptx::mma_commit(&B.s_full[w]);  // the softmax group also frees the K slot on it
-                        if (j == n - 1) ptx::mma_commit(&B.q_empty);
+                        ptx::mma_commit_w(&B.s_full[w]);  // the softmax group also frees the K slot on it
+                        if (j == n - 1) ptx::mma_commit_w(&B.q_empty);
                     }
                 }
             }
@@ -327,12 +331,12 @@ __global__ void __launch_bounds__(384, 1)
             pu[1] += group_tiles(n, 1);
             ++it;
             __syncwarp();
-            if (*abort_flag) break;
+            if (__any_sync(0xffffffffu, *abort_flag)) break;
         }
-        if (lane == 0) {
+        {
             // every MMA issued so far must finish before the TMEM is released
             volatile int never = 0;
-            ptx::mma_commit(&B.drain);
+            ptx::mma_commit_w(&B.drain);
             ptx::mbar_wait(&B.drain, 0, &never, kDrainNs);
         }
     } else if (warp >= 4) {

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(384, 1)
         const bool kq = warp == 0;
         const int S = kq ? KS : VS;
         const uint64_t keep = ptx::policy_evict_last();
-        int issued_q = 0, issued = 0;  // copies issued so far (lane 0): Q tiles; K or V tiles
+        int issued_q = 0, issued = 0;  // copies issued so far (warp-uniform): Q tiles; K or V tiles
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
@@ -227,33 +227,37 @@ __global__ void __launch_bounds__(384, 1)
             if (kq && bad && lane == 0) atomicOr(a.err, kErrBadList);
             if (n == 0) continue;
             const int32_t row0 = int32_t(int64_t(hh) * a.n_slots);
-            if (kq && lane == 0 && !a.hold_q && ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo)) {
-                ptx::mbar_arrive_expect_tx(&B.q_full, C::kQKBytes);
-                for (int x = 0; x < C::kBoxesQK; ++x)
-                    ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * (kFp8 ? 128 : 64), row0 + qt * 128, &B.q_full);
+            if (kq && !a.hold_q &&
+                __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo))) {
+                if (ptx::elect_one()) {
+                    ptx::mbar_arrive_expect_tx(&B.q_full, C::kQKBytes);
+                    for (int x = 0; x < C::kBoxesQK; ++x)
+                        ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * (kFp8 ? 128 : 64), row0 + qt * 128,
+                                         &B.q_full);
+                }
+                __syncwarp();
                 ++issued_q;
             }
-            __syncwarp();
             if (__any_sync(0xffffffffu, *abort_flag)) break;
             int mine = 0;
             for (int j = 0; j < n; ++j) {
                 if ((j & 31) == 0) mine = (j + lane < n) ? __ldg(list + j + lane) : 0;
                 const int y = row0 + __shfl_sync(0xffffffffu, mine, j & 31) * 128;
-                if (lane == 0) {
-                    const int st = issued % S, u = issued / S;
-                    uint64_t* empty = kq ? &B.k_empty[st] : &B.v_empty[st];
-                    uint64_t* full = kq ? &B.k_full[st] : &B.v_full[st];
-                    const int bytes = kq ? C::kQKBytes : C::kTileBytes;
-                    uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * bytes;
-                    if (ptx::mbar_wait(empty, (u & 1) ^ 1, abort_flag, tmo)) {
+                const int st = issued % S, u = issued / S;
+                uint64_t* empty = kq ? &B.k_empty[st] : &B.v_empty[st];
+                uint64_t* full = kq ? &B.k_full[st] : &B.v_full[st];
+                const int bytes = kq ? C::kQKBytes : C::kTileBytes;
+                uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * bytes;
+                if (__all_sync(0xffffffffu, ptx::mbar_wait(empty, (u & 1) ^ 1, abort_flag, tmo))) {
+                    if (ptx::elect_one()) {
                         ptx::mbar_arrive_expect_tx(full, bytes);
                         const int boxes = kq ? C::kBoxesQK : C::kBoxes, xstep = (kq && kFp8) ? 128 : 64;
                         for (int x = 0; x < boxes; ++x)
                             ptx::tma_load_2d_hint(dst + x * 16384, kq ? &tm_k : &tm_v, x * xstep, y, full, keep);
-                        ++issued;
                     }
+                    __syncwarp();
+                    ++issued;
                 }
-                __syncwarp();
                 if (__any_sync(0xffffffffu, *abort_flag)) break;
             }
             if (__any_sync(0xffffffffu, *abort_flag)) break;

@@ -186,6 +186,17 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+// True in exactly one lane of a converged full warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e != 0;
+}
+
 // Warp-uniform forms: the whole (converged) warp executes the call and elect.sync picks the one lane
 // that issues, so operands stay in uniform registers. The elected lane is the same for every call made
 // by a full warp, which keeps the per-thread commit tracking consistent.

@@ -273,8 +273,15 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------------------- MMA issuer (whole warp, one lane issues)
         // Per item: S_0 and S_1, then for each tile j: O_(j%2) += P_j V_j, then S_(j+2). S_j lands in S
         // buffer j%2, which softmax group j%2 turns into P_j in place.
-        int it = 0, t = 0;      // items with tiles so far; tiles so far (ring positions)
-        int pu[2] = {0, 0};     // tiles each group has had so far (barrier phases)
+        int it = 0;              // items with tiles so far
+        int ks = 0, kph = 0;     // K ring slot of the next S and its phase
+        int vs = 0, vph = 0;     // V ring slot of the next PV and its phase
+        int pu[2] = {0, 0};      // tiles each group has had so far (barrier phases)
+        // shared-memory descriptors of the first Q, K and V boxes; a k-step or a ring slot only moves the
+        // start address, which is the descriptor's low field (address / 16, below 2^14 for any CTA address)
+        const uint64_t dq = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffQ), 16, 1024);
+        const uint64_t dk = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffK), 16, 1024);
+        const uint64_t dv = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffV), 16384, 1024);
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
@@ -283,54 +290,54 @@ __global__ void __launch_bounds__(384, 1)
             const int n = item_tiles(a, hh, qt, &list, &bad);
             if (n == 0) continue;
             {
-                const uint32_t q0 = ptx::smem_addr(smem + C::kOffQ);
                 bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_full, it & 1, abort_flag, tmo));
                 for (int j = 0; ok && j < n + 2; ++j) {
                     if (j >= 2) {
                         // O_w += P V for tile jj = j - 2
-                        const int jj = j - 2, w = jj & 1, idx = pu[w] + (jj >> 1), tv = t + jj, sv = tv % VS;
+                        const int jj = j - 2, w = jj & 1, idx = pu[w] + (jj >> 1);
                         ok = ptx::mbar_wait(&B.p_full[w], idx & 1, abort_flag, tmo) &&
-                             ptx::mbar_wait(&B.v_full[sv], (tv / VS) & 1, abort_flag, tmo) &&
+                             ptx::mbar_wait(&B.v_full[vs], vph, abort_flag, tmo) &&
                              (jj > 0 || ptx::mbar_wait(&B.o_empty, (it & 1) ^ 1, abort_flag, tmo));
                         ok = __all_sync(0xffffffffu, ok);
                         if (!ok) break;
                         ptx::tc_fence_after();
-                        const uint32_t v0 = ptx::smem_addr(smem + C::kOffV + sv * C::kTileBytes);
+                        const uint64_t dvs = dv + uint64_t(vs * (C::kTileBytes >> 4));
                         const uint32_t o = tmem + 256 + 128 * w, p = tmem + 128 * w;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            ptx::mma_bf16_ts_w(o, p + kk * 8, ptx::smem_desc_sw128(v0 + kk * 2048, 16384, 1024), C::kIdescPV,
-                                             (jj >= 2 || kk > 0) ? 1u : 0u);
-                        ptx::mma_commit_w(&B.v_empty[sv]);
+                            ptx::mma_bf16_ts_w(o, p + kk * 8, dvs + uint64_t(kk * (2048 >> 4)), C::kIdescPV,
+                                               (jj >= 2 || kk > 0) ? 1u : 0u);
+                        ptx::mma_commit_w(&B.v_empty[vs]);
                         if (jj >= n - 2) ptx::mma_commit_w(&B.o_done[w]);  // the group's last tile of the item
+                        if (++vs == VS) vs = 0, vph ^= 1;
                     }
                     if (j < n) {
                         // S_j = Q K_j^T into S buffer j%2
-                        const int w = j & 1, tk = t + j, st = tk % KS;
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.k_full[st], (tk / KS) & 1, abort_flag, tmo));
+                        const int w = j & 1;
+                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.k_full[ks], kph, abort_flag, tmo));
                         if (!ok) break;
                         ptx::tc_fence_after();
-                        const uint32_t k0 = ptx::smem_addr(smem + C::kOffK + st * C::kQKBytes);
+                        const uint64_t dks = dk + uint64_t(ks * (C::kQKBytes >> 4));
                         if constexpr (kFp8) {
-                            // e4m3: a 128-byte row holds all 128 dims; K = 32 per MMA
+                            // e4m3: a 128-byte row holds all 128 dims; K = 32 per MMA (32 bytes along the row)
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
-                                ptx::mma_f8_ss_w(tmem + 128 * w, ptx::smem_desc_sw128(q0 + kk * 32, 16, 1024),
-                                               ptx::smem_desc_sw128(k0 + kk * 32, 16, 1024), C::kIdescS, kk > 0);
+                                ptx::mma_f8_ss_w(tmem + 128 * w, dq + uint64_t(kk * 2), dks + uint64_t(kk * 2), C::kIdescS,
+                                                 kk > 0);
                         } else {
+                            // K = 16 per MMA: 32 bytes along a 128-byte row, then the next 64-column box (16 KB on)
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
-                                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                                ptx::mma_bf16_ss_w(tmem + 128 * w, ptx::smem_desc_sw128(q0 + off, 16, 1024),
-                                                 ptx::smem_desc_sw128(k0 + off, 16, 1024), C::kIdescS, kk > 0);
+                                const uint64_t off = uint64_t((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
+                                ptx::mma_bf16_ss_w(tmem + 128 * w, dq + off, dks + off, C::kIdescS, kk > 0);
                             }
                         }
                         ptx::mma_commit_w(&B.s_full[w]);  // the softmax group also frees the K slot on it
                         if (j == n - 1) ptx::mma_commit_w(&B.q_empty);
+                        if (++ks == KS) ks = 0, kph ^= 1;
                     }
                 }
             }
-            t += n;
             pu[0] += group_tiles(n, 0);
             pu[1] += group_tiles(n, 1);
             ++it;
@@ -504,6 +511,9 @@ __global__ void __launch_bounds__(384, 1)
             const float inv = den > 0.f ? 1.f / den : 0.f;
             const float s0 = a0 * inv, s1 = a1 * inv;
             ptx::tc_fence_after();
+            // both accumulators' columns of our half are read (and merged into bf16 pairs) before O is
+            // released to the next item's first PV; the global stores come after the release
+            uint32_t res[D / 4];
 #pragma unroll
             for (int i = 0; i < D / 64; ++i) {
                 const uint32_t col = w * (D / 2) + 32 * i;
@@ -511,25 +521,24 @@ __global__ void __launch_bounds__(384, 1)
                 ptx::tmem_ld32(t_o0 + col, o0);
                 ptx::tmem_ld32(t_o0 + 128 + col, o1);
                 ptx::tmem_wait_ld();
-                if (i == D / 64 - 1) {
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(&B.o_empty);
-                }
-                if (prow >= 0) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * i);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float v[8];
+                for (int c = 0; c < 16; ++c) {
+                    float v[2];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float x0 = s0 != 0.f ? __uint_as_float(o0[8 * c + e]) * s0 : 0.f;
-                            const float x1 = s1 != 0.f ? __uint_as_float(o1[8 * c + e]) * s1 : 0.f;
-                            v[e] = x0 + x1;
-                        }
-                        d4[c] = make_uint4(ptx::pack_bf16(v[0], v[1]), ptx::pack_bf16(v[2], v[3]),
-                                           ptx::pack_bf16(v[4], v[5]), ptx::pack_bf16(v[6], v[7]));
+                    for (int u = 0; u < 2; ++u) {
+                        const float x0 = s0 != 0.f ? __uint_as_float(o0[2 * c + u]) * s0 : 0.f;
+                        const float x1 = s1 != 0.f ? __uint_as_float(o1[2 * c + u]) * s1 : 0.f;
+                        v[u] = x0 + x1;
                     }
+                    res[16 * i + c] = ptx::pack_bf16(v[0], v[1]);
                 }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&B.o_empty);
+            if (prow >= 0) {
+                uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c) d4[c] = make_uint4(res[4 * c], res[4 * c + 1], res[4 * c + 2], res[4 * c + 3]);
             }
         }
     }

@@ -132,13 +132,15 @@ def flops_per_pair(dim):
 def stage_bytes(layer, wl):
     """Algorithmic HBM bytes per launch of each stage, summed over head groups."""
     D, S = wl.dim, wl.seq_len
-    out = {"gather_qk": 0, "score": 0, "select": 0, "gather_v": 0, "quantize": 0, "attend": 0}
+    out = {"gather_qk": 0, "score": 0, "select": 0, "gather_v": 0, "attend": 0}
     for g in layer.groups:
         lay, n = g["layout"], len(g["heads_list"])
         real = n * S * D * 2
         slots = n * lay.n_slots * D * 2
         feats = n * lay.n_video * 3 * D * 4
-        out["gather_qk"] += 2 * (real + slots + feats)
+        # the FP8 Q/K variant writes e4m3 codes (1 byte per element) and per-tile scales instead of bf16
+        tiles_out = slots // 2 + n * lay.n_tiles * 4 if layer.fp8_qk else slots
+        out["gather_qk"] += 2 * (real + tiles_out + feats)
         out["gather_v"] += real + slots
         sc = n * lay.n_video * lay.n_video * 4
         proj = 2 * n * 3 * D * D * 4
@@ -146,9 +148,8 @@ def stage_bytes(layer, wl):
         out["score"] += 2 * feats + proj + 2 * hat + sc
         kept = int(g["kept_cnt"].sum())
         out["select"] += sc + 4 * (kept + n * lay.n_video)
-        out["attend"] += slots + real + 4 * (kept + n * lay.n_video)  # Q in, O out, lists; K/V counted as L2 reuse
-        if layer.fp8_qk:
-            out["quantize"] += 2 * (slots + slots // 2)  # bf16 Q and K tiles in, e4m3 codes out
+        q_in = slots // 2 if layer.fp8_qk else slots
+        out["attend"] += q_in + real + 4 * (kept + n * lay.n_video)  # Q in, O out, lists; K/V counted as L2 reuse
     return out
 
 

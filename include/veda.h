@@ -208,6 +208,17 @@ int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, con
 int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim, void* codes,
                       float* scales, void* stream);
 
+/* FP8 Q/K variant, steps 0 and 1 in one pass: veda_gather with the tile written as e4m3 codes and its
+ * per-tile scale (the quantisation of veda_quantize_fp8, bit for bit) instead of bf16, so the bf16 tile
+ * copy is never written or read back.
+ *  x, x_strides, h_total, heads, feats  as veda_gather (feats may be NULL).
+ *  codes   device e4m3 bytes [n_heads, N, D] out (padding slots 0).
+ *  scales  device fp32 [n_heads, n_tiles] out.
+ * D must be 64 or 128. Errors as veda_gather. */
+int veda_gather_fp8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                    int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales, float* feats,
+                    void* stream);
+
 /* FP8 Q/K variant, step 2: veda_attend with Q and K given as e4m3 codes and per-tile scales (from
  * veda_quantize_fp8); S = Q K^T runs as an e4m3 x e4m3 tensor-core product with fp32 accumulation and is
  * multiplied by scale_q(query tile) * scale_k(key tile) * D^-0.5; P and V stay bf16. Selection is not

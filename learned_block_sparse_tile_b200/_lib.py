@@ -21,7 +21,7 @@ EXPORTS = [
     "veda_plan", "veda_layout_info", "veda_layout_export", "veda_layout_destroy", "veda_least_padding_box",
     "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_score_noalloc", "veda_select", "veda_attend",
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
-    "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_attend_fp8",
+    "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
 ]
 
 
@@ -81,6 +81,7 @@ def lib():
         L.veda_select.argtypes = [vp, p, i32, p, p, vp]
         L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_quantize_fp8.argtypes = [vp, p, i32, i32, p, p, vp]
+        L.veda_gather_fp8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
         L.veda_attend_fp8.argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_sync_status.argtypes = [vp]
         L.veda_last_error.restype = C.c_char_p
@@ -204,6 +205,13 @@ def veda_attend(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, stream=No
     _check(lib().veda_attend(layout.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), q_t.shape[0], q_t.shape[2],
                              _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1], _ptr(heads),
                              _stream(stream)))
+
+
+def veda_gather_fp8(layout, x, heads, codes, scales, feats=None, stream=None):
+    """x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; codes: uint8 [n, N, D] (e4m3 bytes); scales: fp32
+    [n, n_tiles]; feats: fp32 [n, n_video, 3D] or None."""
+    _check(lib().veda_gather_fp8(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
+                                 heads.numel(), _ptr(codes), _ptr(scales), _ptr(feats), _stream(stream)))
 
 
 def veda_quantize_fp8(layout, x_t, codes, scales, stream=None):

@@ -20,17 +20,23 @@ struct QuantArgs {
     int32_t n_tiles;
 };
 
-// x / s rounded once to e4m3. The quotient is formed in double and narrowed to fp32 with round-to-odd
-// (truncate, then set the last bit when anything was cut off), so the final round-to-nearest-even into
-// e4m3 (3 mantissa bits, far fewer than fp32's 23) equals rounding the double quotient directly. A plain
-// fp32 division would round twice: quotients of bf16 values by amax / 448 often land within a few ulps of
-// an e4m3 midpoint (for example 42.0000014 between 40 and 44) and the first rounding would move them
-// onto it.
+// x / s rounded once to e4m3. The quotient is narrowed to fp32 with round-to-odd (the truncated quotient,
+// with its last bit set when anything was cut off), so the final round-to-nearest-even into e4m3 (3
+// mantissa bits, far fewer than fp32's 23) equals rounding the exact quotient directly. A plain fp32
+// division would round twice: quotients of bf16 values by amax / 448 often land within a few ulps of an
+// e4m3 midpoint (for example 42.0000014 between 40 and 44) and the first rounding would move them onto it.
+// Round-to-odd from the correctly rounded fp32 quotient q: the residual x - q s is exactly representable
+// in fp32 (a property of round-to-nearest division when nothing underflows) and one FMA gives it; its
+// sign says on which side of q the exact quotient lies (s > 0). When |x / s| > |q| the truncation is q,
+// otherwise it is q one unit lower in magnitude; either way the inexact result is that value with its
+// last bit set. Quotients small enough to underflow round to 0 in e4m3 whatever happens here.
 __device__ __forceinline__ float quotient_round_odd(float x, float s) {
-    const double q = double(x) / double(s);
-    float r = __double2float_rz(q);
-    if (double(r) != q) r = __int_as_float(__float_as_int(r) | 1);
-    return r;
+    const float q = __fdiv_rn(x, s);
+    const float r = fmaf(-q, s, x);
+    if (r == 0.f || q == 0.f) return q;
+    const uint32_t b = __float_as_uint(q), sign = b & 0x80000000u, mag = b & 0x7fffffffu;
+    const bool away = (r > 0.f) == (q > 0.f);  // the exact quotient is larger in magnitude than q
+    return __uint_as_float(sign | ((away ? mag : mag - 1u) | 1u));
 }
 
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
@@ -39,8 +45,54 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return r;
 }
 
-// One CTA per (tile, head), 256 threads; D / 8 threads cover a row (16 bytes each) and each thread keeps its
-// 8 values of 128 / (256 / (D / 8)) rows in registers between the amax pass and the conversion pass.
+// Quantises one (head, 128-row tile) held by a 256-thread CTA: D / 8 threads cover a row (8 bf16 = 16
+// bytes each), thread tid holds rows r0 + p * kRpp (r0 = tid / (D / 8)) of its 8 columns in v[p]. Rows
+// from vc on are padding (zero, and left out of the amax). Writes the tile's scale (thread 0) and the
+// codes of all 128 rows to codes (this thread's column chunk of row 0; rows are D bytes apart). Contains a
+// block barrier: every thread of the CTA must call it.
+template <int D>
+__device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, float* red8, uint8_t* codes,
+                                              float* scale) {
+    constexpr int kTpr = D / 8;
+    constexpr int kRpp = 256 / kTpr;
+    constexpr int kPasses = 128 / kRpp;
+    float amax = 0.f;
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        if (r0 + p * kRpp < vc) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if ((threadIdx.x & 31) == 0) red8[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    float m = red8[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red8[w]);
+    const float s = m > 0.f ? m / 448.f : 1.f;
+    if (threadIdx.x == 0) *scale = s;
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
+        uint32_t w[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
+            w[e] = uint32_t(e4m3x2(quotient_round_odd(f0.x, s), quotient_round_odd(f0.y, s))) |
+                   (uint32_t(e4m3x2(quotient_round_odd(f1.x, s), quotient_round_odd(f1.y, s))) << 16);
+        }
+        *reinterpret_cast<uint2*>(codes + int64_t(r0 + p * kRpp) * D) = make_uint2(w[0], w[1]);
+    }
+}
+
+// One CTA per (tile, head), 256 threads, over a tile-ordered bf16 tensor. HBM bound: reads 2 bytes and
+// writes 1 byte per element.
 template <int D>
 __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
     constexpr int kTpr = D / 8;
@@ -52,42 +104,9 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
     const int vc = __ldg(a.valid_count + tile);
     const int64_t base = (int64_t(hh) * a.n_slots + int64_t(tile) * 128) * D + c * 8;
     uint4 v[kPasses];
-    float amax = 0.f;
 #pragma unroll
-    for (int p = 0; p < kPasses; ++p) {
-        const int r = r0 + p * kRpp;
-        v[p] = *reinterpret_cast<const uint4*>(a.x_t + base + int64_t(r) * D);
-        if (r < vc) {
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-        }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if ((tid & 31) == 0) red[tid >> 5] = amax;
-    __syncthreads();
-    float m = red[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
-    const float s = m > 0.f ? m / 448.f : 1.f;
-    if (tid == 0) a.scales[int64_t(hh) * a.n_tiles + tile] = s;
-#pragma unroll
-    for (int p = 0; p < kPasses; ++p) {
-        const int r = r0 + p * kRpp;
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
-        uint32_t w[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
-            w[e] = uint32_t(e4m3x2(quotient_round_odd(f0.x, s), quotient_round_odd(f0.y, s))) |
-                   (uint32_t(e4m3x2(quotient_round_odd(f1.x, s), quotient_round_odd(f1.y, s))) << 16);
-        }
-        *reinterpret_cast<uint2*>(a.codes + base + int64_t(r) * D) = make_uint2(w[0], w[1]);
-    }
+    for (int p = 0; p < kPasses; ++p) v[p] = *reinterpret_cast<const uint4*>(a.x_t + base + int64_t(r0 + p * kRpp) * D);
+    quantize_tile<D>(v, r0, vc, red, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
 }
 
 }  // namespace veda

@@ -202,6 +202,9 @@ extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64
     a.perm = dc->perm;
     a.valid_count = dc->valid_count;
     a.x_t = static_cast<__nv_bfloat16*>(x_t);
+    a.codes = nullptr;
+    a.scales = nullptr;
+    a.n_tiles = d.n_tiles;
     a.feats = feats;
     a.n_slots = d.n_slots;
     a.n_video = d.n_video;
@@ -214,6 +217,46 @@ extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64
     else
         gather_pool_kernel<64><<<grid, 256, 0, s>>>(a);
     return launch_check("gather_pool_kernel");
+}
+
+extern "C" int veda_gather_fp8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                               int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales,
+                               float* feats, void* stream) {
+    clear_error();
+    if (!layout || !x || !heads || !codes || !scales) return fail(VEDA_ERR_INVALID, "veda_gather_fp8: NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_gather_fp8: head_dim must be 64 or 128");
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_gather_fp8: head counts must be positive");
+    if (int rc = check_strided(x_strides, x, "veda_gather_fp8 x")) return rc;
+    if (!aligned16(codes) || !aligned16(scales) || (feats && !aligned16(feats)))
+        return fail(VEDA_ERR_INVALID, "veda_gather_fp8: outputs need 16-byte alignment");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    const veda_layout_desc& d = layout->desc;
+    GatherArgs a;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.s0 = x_strides[0];
+    a.s1 = x_strides[1];
+    a.heads = heads;
+    a.perm = dc->perm;
+    a.valid_count = dc->valid_count;
+    a.x_t = nullptr;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.n_tiles = d.n_tiles;
+    a.feats = feats;
+    a.n_slots = d.n_slots;
+    a.n_video = d.n_video;
+    a.h_total = h_total;
+    a.err = ds->err;
+    dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dim == 128)
+        gather_pool_kernel<128, true><<<grid, 256, 0, s>>>(a);
+    else
+        gather_pool_kernel<64, true><<<grid, 256, 0, s>>>(a);
+    return launch_check("gather_pool_kernel (e4m3 codes)");
 }
 
 extern "C" size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim) {

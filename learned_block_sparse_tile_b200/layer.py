@@ -1,8 +1,9 @@
 """One Veda attention layer on the C ABI (veda_core.py, "one layer", attention).
 
 For each group of heads sharing a target tile box: plan (cached), gather Q and K to tile order with
-pooling, score, select, gather V, attend with the scatter fused. PyTorch only allocates device buffers
-and supplies the stream; every step runs in libveda's kernels.
+pooling (straight to e4m3 codes and per-tile scales in the FP8 Q/K variant), score, select, gather V,
+attend with the scatter fused. PyTorch only allocates device buffers and supplies the stream; every step
+runs in libveda's kernels.
 """
 from __future__ import annotations
 
@@ -41,8 +42,6 @@ class VedaLayer:
             dev = self.device
             g = dict(box=box, heads_list=hs, layout=lay,
                      heads=torch.tensor(hs, dtype=torch.int32, device=dev),
-                     q_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
-                     k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
                      v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
                      feats_q=torch.empty(n, lay.n_video, 3 * dim, dtype=torch.float32, device=dev),
                      feats_k=torch.empty(n, lay.n_video, 3 * dim, dtype=torch.float32, device=dev),
@@ -51,13 +50,16 @@ class VedaLayer:
                      scores=torch.empty(n, lay.n_video, lay.n_video, dtype=torch.float32, device=dev),
                      kept_idx=torch.empty(n, lay.n_video, lay.max_kept, dtype=torch.int32, device=dev),
                      kept_cnt=torch.empty(n, lay.n_video, dtype=torch.int32, device=dev))
-            if self.fp8_qk:
+            if self.fp8_qk:  # Q and K are gathered straight to e4m3 codes with per-tile scales
                 g.update(q8=torch.empty(n, lay.n_slots, dim, dtype=torch.uint8, device=dev),
                          k8=torch.empty(n, lay.n_slots, dim, dtype=torch.uint8, device=dev),
                          sq=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev),
                          sk=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev))
+            else:
+                g.update(q_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
+                         k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
             self.groups.append(g)
-        self.launches = (self.LAUNCHES_PER_GROUP + 2 * self.fp8_qk) * len(self.groups)
+        self.launches = self.LAUNCHES_PER_GROUP * len(self.groups)
 
     def set_projections(self, proj_q, proj_k):
         """proj_q, proj_k: fp32 [H, 3D, D] (any device); each group keeps its heads' slices on device."""
@@ -92,8 +94,7 @@ class VedaLayer:
         """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten.
 
         ``events``: optional dict; CUDA event pairs recorded around each stage on ``stream`` are appended
-        under the stage names gather_qk, score, select, gather_v, quantize (FP8 Q/K only) and attend (the
-        page's PhaseTimer)."""
+        under the stage names gather_qk, score, select, gather_v and attend (the page's PhaseTimer)."""
         st = stream if stream is not None else torch.cuda.current_stream()
 
         def mark(name):
@@ -113,8 +114,12 @@ class VedaLayer:
         for g in self.groups:
             lay = g["layout"]
             m = mark("gather_qk")
-            L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st)
-            L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st)
+            if self.fp8_qk:
+                L.veda_gather_fp8(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st)
+                L.veda_gather_fp8(lay, k, g["heads"], g["k8"], g["sk"], g["feats_k"], st)
+            else:
+                L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st)
+                L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st)
             done(m)
             m = mark("score")
             L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"], st)
@@ -126,10 +131,6 @@ class VedaLayer:
             L.veda_gather(lay, v, g["heads"], g["v_t"], None, st)
             done(m)
             if self.fp8_qk:
-                m = mark("quantize")
-                L.veda_quantize_fp8(lay, g["q_t"], g["q8"], g["sq"], st)
-                L.veda_quantize_fp8(lay, g["k_t"], g["k8"], g["sk"], st)
-                done(m)
                 m = mark("attend")
                 L.veda_attend_fp8(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"],
                                   out, g["heads"], st)

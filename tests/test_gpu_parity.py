@@ -191,3 +191,31 @@ def test_fp8_qk_variant():
     mx, _ = attention_error(got, want_ref)
     q_err, _ = attention_error(want_fp8, want_ref)
     assert mx <= q_err + ATT_MAX_ABS, (mx, q_err)
+
+
+@pytest.mark.parametrize("name", ["small_d128", "padded_tiny", "small_mixed"])
+def test_fused_fp8_gather(name):
+    # gather straight to e4m3 codes: codes and scales equal the two-pass path (gather, then quantise) and
+    # the oracle's reading bit for bit, on head_dim 128 and 64, padded tiles and global tiles; the pooled
+    # features equal the bf16 gather's
+    c = case(name)
+    wl = c.wl
+    for box, heads in c.groups:
+        res = c.run_group(box, heads)
+        lay = res["layout"]
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        n = len(heads)
+        for x, x_t, f_ref in ((c.dq, res["q_t"], res["fq"]), (c.dk, res["k_t"], res["fk"])):
+            codes = torch.full((n, lay.n_slots, wl.dim), 0x55, dtype=torch.uint8, device="cuda")
+            scales = torch.full((n, lay.n_tiles), -1.0, dtype=torch.float32, device="cuda")
+            feats = torch.full_like(f_ref, float("nan"))
+            L.veda_gather_fp8(lay, x, res["heads"], codes, scales, feats)
+            codes2, scales2 = torch.empty_like(codes), torch.empty_like(scales)
+            L.veda_quantize_fp8(lay, x_t, codes2, scales2)
+            assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+            assert torch.equal(codes, codes2) and torch.equal(scales, scales2)
+            assert torch.equal(feats, f_ref)
+            want_codes, want_scales = O.quantize_fp8_tiles(O.gather(f32(x), lay_o, heads), lay_o)
+            assert np.array_equal(f32(scales).astype(np.float64), want_scales)
+            got = codes.view(torch.float8_e4m3fn).float().cpu().numpy().transpose(1, 0, 2)
+            assert np.array_equal(got, want_codes)

@@ -25,13 +25,16 @@ struct QuantArgs {
 // mantissa bits, far fewer than fp32's 23) equals rounding the exact quotient directly. A plain fp32
 // division would round twice: quotients of bf16 values by amax / 448 often land within a few ulps of an
 // e4m3 midpoint (for example 42.0000014 between 40 and 44) and the first rounding would move them onto it.
-// Round-to-odd from the correctly rounded fp32 quotient q: the residual x - q s is exactly representable
-// in fp32 (a property of round-to-nearest division when nothing underflows) and one FMA gives it; its
-// sign says on which side of q the exact quotient lies (s > 0). When |x / s| > |q| the truncation is q,
-// otherwise it is q one unit lower in magnitude; either way the inexact result is that value with its
+//
+// Round-to-odd needs only a faithful quotient q (one of the two fp32 neighbours of x / s) and the side of
+// q on which x / s lies. q: x times the tile's reciprocal inv = 1/s, refined once by the FMA residual
+// (q0 + (x - q0 s) inv is within one unit of x / s). The side: the sign of x - q s, formed exactly inside
+// one FMA and rounded once, which keeps its sign and its being zero (s > 0). When |x / s| > |q| the
+// truncation is q, otherwise q one unit lower in magnitude; the inexact result is that value with its
 // last bit set. Quotients small enough to underflow round to 0 in e4m3 whatever happens here.
-__device__ __forceinline__ float quotient_round_odd(float x, float s) {
-    const float q = __fdiv_rn(x, s);
+__device__ __forceinline__ float quotient_round_odd(float x, float s, float inv) {
+    const float q0 = x * inv;
+    const float q = fmaf(fmaf(-q0, s, x), inv, q0);
     const float r = fmaf(-q, s, x);
     if (r == 0.f || q == 0.f) return q;
     const uint32_t b = __float_as_uint(q), sign = b & 0x80000000u, mag = b & 0x7fffffffu;
@@ -76,6 +79,7 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
 #pragma unroll
     for (int w = 1; w < 8; ++w) m = fmaxf(m, red8[w]);
     const float s = m > 0.f ? m / 448.f : 1.f;
+    const float inv = 1.f / s;
     if (threadIdx.x == 0) *scale = s;
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
@@ -84,8 +88,8 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
-            w[e] = uint32_t(e4m3x2(quotient_round_odd(f0.x, s), quotient_round_odd(f0.y, s))) |
-                   (uint32_t(e4m3x2(quotient_round_odd(f1.x, s), quotient_round_odd(f1.y, s))) << 16);
+            w[e] = uint32_t(e4m3x2(quotient_round_odd(f0.x, s, inv), quotient_round_odd(f0.y, s, inv))) |
+                   (uint32_t(e4m3x2(quotient_round_odd(f1.x, s, inv), quotient_round_odd(f1.y, s, inv))) << 16);
         }
         *reinterpret_cast<uint2*>(codes + int64_t(r0 + p * kRpp) * D) = make_uint2(w[0], w[1]);
     }

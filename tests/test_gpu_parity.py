@@ -219,3 +219,68 @@ def test_fused_fp8_gather(name):
             assert np.array_equal(f32(scales).astype(np.float64), want_scales)
             got = codes.view(torch.float8_e4m3fn).float().cpu().numpy().transpose(1, 0, 2)
             assert np.array_equal(got, want_codes)
+
+
+def _bf16(x):
+    """float64 values that are exactly bf16 -> bf16 bit patterns (uint16)."""
+    b = np.asarray(x, dtype=np.float32).view(np.uint32)
+    assert np.all(b & 0xFFFF == 0), "value not representable in bf16"
+    return (b >> 16).astype(np.uint16)
+
+
+def _midpoint_tile(rng, mode, D):
+    """One 128 x D tile of bf16 bits whose quotients by the tile's fp32 scale sit on e4m3 rounding
+    midpoints. mode 'near': amax has at most 6 significant bits and is not a multiple of 7, so
+    amax / 448 is inexact in fp32; x = 3 amax 2^(j-9) is exact in bf16 and x / (amax / 448) is exactly the
+    midpoint 2.625 2^j (and amax 2^-16 gives the subnormal midpoint 7 2^-10): the rounding of the stored
+    scale alone moves x / s off the midpoint, by less than one fp32 ulp. mode 'tie': the scale is a power of
+    two and every e4m3 midpoint times it is exact, so x / s is exactly a midpoint (ties to even)."""
+    vals = np.array([float(v) for v in torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).float()])
+    mids = (vals[:-1] + vals[1:]) / 2
+    if mode == "near":
+        amax = float(rng.choice([13.0, 5.75, 27.5, 1.5, 0.8125, 19.0, 43.0, 2.75]))
+        xs = np.concatenate([3 * amax * 2.0 ** (np.arange(-6, 8) - 9), [amax * 2.0 ** -16]])
+    else:
+        k = int(rng.integers(1, 6))
+        amax = 448.0 * 2.0 ** -k
+        xs = mids * 2.0 ** -k
+    xs = xs[xs < amax]
+    bits = _bf16(np.concatenate([xs, -xs]))
+    tile = rng.choice(bits, size=(128, D))
+    tile[0, 0] = _bf16([amax])[0]
+    return tile
+
+
+def test_fp8_codes_at_rounding_midpoints():
+    # quotients within one fp32 ulp of (or exactly on) e4m3 rounding midpoints: the quantiser's
+    # round-to-odd quotient must round like the exact quotient. Standalone quantiser and fused gather,
+    # against the oracle bit for bit.
+    c = case("padded_tiny")
+    wl = c.wl
+    box, heads = c.groups[0]
+    lay = c.run_group(box, heads)["layout"]
+    lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+    D, N = wl.dim, lay.n_slots
+    rng = np.random.default_rng(11)
+    bits = np.zeros((N, D), dtype=np.uint16)
+    for i in range(lay.n_tiles):
+        tile = _midpoint_tile(rng, "near" if i % 3 else "tie", D)
+        tile[int(lay_o.valid_count[i]):] = 0  # padding slots are zero
+        bits[i * 128:(i + 1) * 128] = tile
+    x_t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(1, N, D).cuda()
+    codes = torch.empty(1, N, D, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(1, lay.n_tiles, dtype=torch.float32, device="cuda")
+    L.veda_quantize_fp8(lay, x_t, codes, scales)
+    # the same tiles through the fused gather: scatter them back to packed rows first
+    perm = lay_o.perm
+    real = np.flatnonzero(perm >= 0)
+    x = torch.zeros(wl.seq_len, 1, D, dtype=torch.bfloat16)
+    x[torch.from_numpy(perm[real]).long(), 0] = x_t[0].cpu()[torch.from_numpy(real).long()]
+    codes_g, scales_g = torch.empty_like(codes), torch.empty_like(scales)
+    L.veda_gather_fp8(lay, x.cuda(), torch.zeros(1, dtype=torch.int32, device="cuda"), codes_g, scales_g)
+    assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+    want_codes, want_scales = O.quantize_fp8_tiles(f32(x_t).transpose(1, 0, 2), lay_o)
+    for cd, sc in ((codes, scales), (codes_g, scales_g)):
+        assert np.array_equal(f32(sc).astype(np.float64), want_scales)
+        got = cd.view(torch.float8_e4m3fn).float().cpu().numpy().transpose(1, 0, 2)
+        assert np.array_equal(got, want_codes), int((got != want_codes).sum())

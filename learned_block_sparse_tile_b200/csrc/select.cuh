@@ -204,4 +204,101 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectArgs
     if (tid == 0) a.kept_cnt[rowid] = pos + a.n_global_ok;
 }
 
+// The same selection with one warp per (video query row, head), for column blocks of at most 32 kPer
+// tiles. Column c of a block sits in lane c % 32, slot c / 32, so ballots over a slot list columns in
+// ascending order. The threshold key T (the allowed-th largest key of the block) is built bit by bit from
+// the top: a candidate bit stays set when at least `allowed` keys are >= the candidate (when exactly
+// `allowed` are, T is the smallest of them and the search stops). Keys above T are
+// kept, and of the keys equal to T the lowest columns, as many as are still needed. No shared memory and
+// no block barriers: a warp owns its row.
+template <int kPer>
+__global__ void __launch_bounds__(256) select_warp_kernel(const SelectArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), hh = blockIdx.y;
+    if (row >= a.n_video) return;  // whole warps only
+    const unsigned lower = (1u << lane) - 1u;
+    const int64_t rowid = int64_t(hh) * a.n_video + row;
+    const float* srow = a.scores + rowid * a.n_video;
+    int32_t* out = a.kept_idx + rowid * a.max_kept;
+    int pos = 0;
+    for (int b = 0; b < a.n_blocks; ++b) {
+        const int start = a.blk_start[b], n = a.blk_stop[b] - start;
+        if (a.blk_all[b]) {
+            for (int i = 0; i * 32 < n; ++i) {
+                const int c = i * 32 + lane;
+                const bool ok = c < n && __ldg(a.valid_count + start + c) > 0;
+                const unsigned bal = __ballot_sync(0xffffffffu, ok);
+                if (ok) out[pos + __popc(bal & lower)] = start + c;
+                pos += __popc(bal);
+            }
+            continue;
+        }
+        const int allowed = __ldg(a.allowed + int64_t(b) * a.n_video + row);
+        uint32_t key[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int c = i * 32 + lane, col = start + c;
+            uint32_t k = 0;  // below every real key (the -inf key is 0x007FFFFF); never counted or kept
+            if (c < n) {
+                k = order_key(__ldg(srow + col));
+                if (__ldg(a.valid_count + col) <= 0) k = kKeyNeg;
+                if (col == row) k = kKeyPos;
+            }
+            key[i] = k;
+        }
+        uint32_t thr;  // keep keys > thr, plus the first `need` keys == thr (lowest columns)
+        int need = 0;
+        if (allowed <= 0) {
+            thr = 0xFFFFFFFFu;  // nothing is kept
+        } else if (allowed >= n) {
+            thr = 0u;  // every real key is > 0
+        } else {
+            // thr keeps at least `allowed` keys >= thr. A candidate with exactly `allowed` keys >= it ends the
+            // search: the allowed-th largest key is then the smallest of those keys.
+            thr = 0u;
+            bool exact = false;
+            for (int bit = 31; bit >= 0; --bit) {
+                const uint32_t cand = thr | (1u << bit);
+                unsigned cnt = 0;
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) cnt += key[i] >= cand;
+                const int total = int(__reduce_add_sync(0xffffffffu, cnt));
+                if (total >= allowed) {
+                    thr = cand;
+                    if (total == allowed) {
+                        exact = true;
+                        break;
+                    }
+                }
+            }
+            if (exact) {
+                uint32_t lo = 0xFFFFFFFFu;
+#pragma unroll
+                for (int i = 0; i < kPer; ++i)
+                    if (key[i] >= thr) lo = min(lo, key[i]);
+                thr = __reduce_min_sync(0xffffffffu, lo);
+            }
+            unsigned above = 0;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) above += key[i] > thr;
+            need = allowed - int(__reduce_add_sync(0xffffffffu, above));
+        }
+        int ties = 0;  // keys == thr taken so far, in column order
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const uint32_t k = key[i];
+            const unsigned tie = __ballot_sync(0xffffffffu, k == thr && thr != 0u);
+            const bool take = k != 0u && k != kKeyNeg &&
+                              (k > thr || (k == thr && ties + __popc(tie & lower) < need));
+            ties += __popc(tie);
+            const unsigned bal = __ballot_sync(0xffffffffu, take);
+            if (take) out[pos + __popc(bal & lower)] = start + i * 32 + lane;
+            pos += __popc(bal);
+        }
+    }
+    const int* glob = a.ok_list + (a.n_kv_ok - a.n_global_ok);
+    for (int i = lane; i < a.n_global_ok; i += 32) out[pos + i] = __ldg(glob + i);
+    if (lane == 0) a.kept_cnt[rowid] = pos + a.n_global_ok;
+}
+
 }  // namespace veda

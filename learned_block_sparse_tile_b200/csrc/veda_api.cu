@@ -343,6 +343,18 @@ extern "C" int veda_select(const veda_layout* layout, const float* scores, int32
         a.blk_stop[b] = b < d.n_blocks ? d.blocks[b].stop : 0;
         a.blk_all[b] = b < d.n_blocks ? d.blocks[b].keeps_all : 0;
     }
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (widest <= 32 * 64) {
+        // one warp per row, the block's keys in registers
+        const dim3 grid(unsigned((d.n_video + 7) / 8), unsigned(n_heads));
+        if (widest <= 32 * 16)
+            select_warp_kernel<16><<<grid, 256, 0, st>>>(a);
+        else if (widest <= 32 * 32)
+            select_warp_kernel<32><<<grid, 256, 0, st>>>(a);
+        else
+            select_warp_kernel<64><<<grid, 256, 0, st>>>(a);
+        return launch_check("select_warp_kernel");
+    }
     const size_t smem = size_t(widest) * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

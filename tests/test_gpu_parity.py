@@ -284,3 +284,27 @@ def test_fp8_codes_at_rounding_midpoints():
         assert np.array_equal(f32(sc).astype(np.float64), want_scales)
         got = cd.view(torch.float8_e4m3fn).float().cpu().numpy().transpose(1, 0, 2)
         assert np.array_equal(got, want_codes), int((got != want_codes).sum())
+
+
+@pytest.mark.parametrize("width", [512, 513, 1024, 2048, 2049])
+def test_select_block_widths(width):
+    # one video span of exactly `width` tiles: the warp-per-row select at the edges of its register
+    # tiers (16 / 32 / 64 keys per lane) and the CTA-per-row select beyond 2048 columns; scores with
+    # many ties, -inf and NaN, bit for bit against the oracle
+    spans = [(0, (1, 8, 16 * width), (1, 8, 16))]
+    seq_len = 128 * width
+    gen, ref = (0.1, None), (1.0, None)
+    lay = L.veda_plan(spans, seq_len, gen, ref)
+    lay_o = O.build_layout(spans, seq_len)
+    assert lay.n_video == width
+    rng = np.random.default_rng(width)
+    s = np.round(rng.standard_normal((1, width, width)) * 3).astype(np.float32)  # small integers: ties
+    s[0, :, rng.integers(0, width, 7)] = -np.inf
+    s[0, ::5, rng.integers(0, width, 3)] = np.nan
+    scores = torch.from_numpy(s).cuda()
+    idx = torch.full((1, width, lay.max_kept), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, width, dtype=torch.int32, device="cuda")
+    L.veda_select(lay, scores, idx, cnt)
+    assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+    _, mask = oracle_kept(lay_o, s, O.column_blocks(lay_o, gen, ref))
+    compare_lists(dict(kept_idx=idx, kept_cnt=cnt), mask, lay_o)

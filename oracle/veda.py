@@ -28,7 +28,7 @@ __all__ = [
     "least_padding_shape", "span_tiles", "build_layout", "gather", "scatter", "pool", "logits",
     "column_blocks", "allowed_per_row", "select", "block_mask", "tile_index_list", "attend_tiles",
     "attend_dense_mask", "dense_attention", "attention_layer", "work_stats", "quantize_fp8_tiles",
-    "attend_tiles_fp8", "layer_spans",
+    "attend_tiles_fp8", "quantize_int8_tiles", "attend_tiles_int8", "layer_spans",
 ]
 
 
@@ -533,6 +533,57 @@ def attend_tiles_fp8(q_t, k_t, v_t, lay, kept_lists, q_tiles=None):
     """
     cq, sq = quantize_fp8_tiles(q_t, lay)
     ck, sk = quantize_fp8_tiles(k_t, lay)
+    tile_of = np.arange(q_t.shape[0]) // TILE
+    qd = cq * sq.T[tile_of][:, :, None]
+    kd = ck * sk.T[tile_of][:, :, None]
+    return attend_tiles(qd, kd, v_t, lay, kept_lists, q_tiles=q_tiles)
+
+
+# ---------------------------------------------------------------------------------------------------
+# INT8 Q/K variant. The pages' own kernel computes Q K^T in INT8 (a SageAttention-derived Triton
+# kernel) but does not print its quantisation recipe; the reading here is the plainest symmetric one, the
+# FP8 reading's twin: per (head, 128-row tile) scale amax(|x| over real rows) / 127 (1.0 when 0), kept
+# as fp32; codes are x / scale rounded to the nearest integer, ties to even, saturating at +-127.
+# ---------------------------------------------------------------------------------------------------
+
+I8_MAX = 127.0
+
+
+def _round_int8(x):
+    """Round float64 values to the nearest integer (ties to even), saturating at +-127."""
+    return np.clip(np.round(np.asarray(x, dtype=np.float64)), -I8_MAX, I8_MAX)  # numpy rounds half to even
+
+
+def quantize_int8_tiles(x_t, lay):
+    """Per (head, 128-row tile) INT8 quantisation of tile-ordered ``[N, H', D]`` values.
+
+    Returns ``(codes as float64 integers [N, H', D], scales [H', n_tiles] float64)``; the dequantised
+    value is ``code * scale``. Padding rows are zero and stay zero.
+    """
+    n = lay.n_tiles
+    n_heads = x_t.shape[1]
+    scales = np.ones((n_heads, n), dtype=np.float64)
+    codes = np.zeros(x_t.shape, dtype=np.float64)
+    for i in range(n):
+        c = int(lay.valid_count[i])
+        blk = x_t[i * TILE:(i + 1) * TILE].astype(np.float64)
+        for h in range(n_heads):
+            amax = np.abs(blk[:c, h, :]).max() if c else 0.0
+            s = amax / I8_MAX if amax > 0 else 1.0
+            s = float(np.float32(s))  # the scale is stored as fp32
+            scales[h, i] = s
+            codes[i * TILE:(i + 1) * TILE, h, :] = _round_int8(blk[:, h, :] / s)
+    return codes, scales
+
+
+def attend_tiles_int8(q_t, k_t, v_t, lay, kept_lists, q_tiles=None):
+    """Attention with Q and K replaced by their per-tile INT8 quantisation (dequantised exactly).
+
+    The scores are ``(code_q * s_q) . (code_k * s_k) * D**-0.5``, that is the integer dot product of
+    the codes times ``s_q * s_k * D**-0.5``; V stays as given.
+    """
+    cq, sq = quantize_int8_tiles(q_t, lay)
+    ck, sk = quantize_int8_tiles(k_t, lay)
     tile_of = np.arange(q_t.shape[0]) // TILE
     qd = cq * sq.T[tile_of][:, :, None]
     kd = ck * sk.T[tile_of][:, :, None]

@@ -399,6 +399,60 @@ def test_fp8_tile_scales():
     assert np.median(rel) < 0.05
 
 
+# ------------------------------------------------------------------------------------------ INT8 reading
+
+def test_int8_rounding_table():
+    # nearest integer, ties to even, saturating at +-127 (values worked by hand)
+    x = np.array([0.0, 0.49, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.7, -3.7, 126.5, 127.49, 127.5, 300.0, -1e9])
+    want = [0.0, 0.0, 0.0, 2.0, 2.0, -0.0, -2.0, -2.0, 4.0, -4.0, 126.0, 127.0, 127.0, 127.0, -127.0]
+    assert O.veda._round_int8(x).tolist() == want
+
+
+def test_int8_tile_scales_and_rounding_bound():
+    lay = O.build_layout([(0, (3, 10, 12), (2, 8, 8))], 360)
+    rng = np.random.default_rng(13)
+    x = (rng.standard_normal((360, 2, 16)) * 3).astype(np.float32)
+    xt = O.gather(x, lay, [0, 1])
+    codes, scales = O.quantize_int8_tiles(xt, lay)
+    assert np.array_equal(codes, np.round(codes)) and np.abs(codes).max() <= 127
+    tile_of = np.arange(lay.n_tiles * 128) // 128
+    for i in range(lay.n_tiles):
+        for h in range(2):
+            c = lay.valid_count[i]
+            assert np.abs(codes[i * 128:i * 128 + c, h]).max() == 127  # the amax lands on 127
+            amax = np.abs(xt[i * 128:i * 128 + c, h]).max()
+            assert scales[h, i] == float(np.float32(amax / 127.0))
+    # a rounded code is within half a step of the value
+    deq = codes * scales.T[tile_of][:, :, None]
+    step = scales.T[tile_of][:, :, None] * np.ones_like(xt)
+    assert np.all(np.abs(deq - xt)[lay.slot_valid] <= 0.5 * step[lay.slot_valid] * (1 + 1e-6))
+    assert (codes[~lay.slot_valid] == 0).all()
+
+
+def test_int8_attention_exact_on_grid_values():
+    # values that are integer multiples of a power of two with the tile's amax at 127 steps quantise
+    # exactly, so the INT8 reading's attention equals plain attention; different steps per tile and head
+    # catch a scale taken from the wrong tile or head
+    lay = O.build_layout([(0, (3, 10, 12), (2, 8, 8))], 360)
+    rng = np.random.default_rng(14)
+    H, D = 2, 16
+    qt = np.zeros((lay.n_tiles * 128, H, D))
+    kt = np.zeros_like(qt)
+    for arr in (qt, kt):
+        for i in range(lay.n_tiles):
+            c = lay.valid_count[i]
+            for h in range(H):
+                step = 2.0 ** -int(rng.integers(3, 9))
+                blk = rng.integers(-127, 128, size=(c, D)).astype(np.float64)
+                blk[0, 0] = 127 * (1 if rng.random() < 0.5 else -1)
+                arr[i * 128:i * 128 + c, h] = blk * step
+    vt = rng.standard_normal(qt.shape) * lay.slot_valid[:, None, None]
+    lists = lambda hh, i: np.arange(lay.n_tiles)
+    want = O.attend_tiles(qt, kt, vt, lay, lists)
+    got = O.attend_tiles_int8(qt, kt, vt, lay, lists)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
 # ------------------------------------------------------------------------------------------ work counter
 
 def test_work_fraction_plausible_against_printed_report():

@@ -139,7 +139,8 @@ def stage_bytes(layer, wl):
         slots = n * lay.n_slots * D * 2
         feats = n * lay.n_video * 3 * D * 4
         # the FP8 Q/K variant writes e4m3 codes (1 byte per element) and per-tile scales instead of bf16
-        tiles_out = slots // 2 + n * lay.n_tiles * 4 if layer.fp8_qk else slots
+        eight_bit = layer.fp8_qk or layer.int8_qk
+        tiles_out = slots // 2 + n * lay.n_tiles * 4 if eight_bit else slots
         out["gather_qk"] += 2 * (real + tiles_out + feats)
         out["gather_v"] += real + slots
         sc = n * lay.n_video * lay.n_video * 4
@@ -148,7 +149,7 @@ def stage_bytes(layer, wl):
         out["score"] += 2 * feats + proj + 2 * hat + sc
         kept = int(g["kept_cnt"].sum())
         out["select"] += sc + 4 * (kept + n * lay.n_video)
-        q_in = slots // 2 if layer.fp8_qk else slots
+        q_in = slots // 2 if eight_bit else slots
         out["attend"] += q_in + real + 4 * (kept + n * lay.n_video)  # Q in, O out, lists; K/V counted as L2 reuse
     return out
 
@@ -163,7 +164,7 @@ def run_veda(args, rank, world, local):
     q, k, v = V.make_qkv(wl)
     pq, pk = V.make_projections(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk)
+                      wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk)
     layer.set_projections(pq, pk)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     out = torch.empty_like(dq)
@@ -234,7 +235,7 @@ def run_veda(args, rank, world, local):
         "metric": METRIC, "value": round(ms_step / world, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 Q/K, bf16 P/V" if wl.fp8_qk else "bf16",
+        "dtype": "e4m3 Q/K, bf16 P/V" if wl.fp8_qk else "int8 Q/K, bf16 P/V" if wl.int8_qk else "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V with a low-rank locality bias; random predictor projections)",
         "config": {"workload": f"{wl.name}: {wl.note}", "seq_len": wl.seq_len, "heads": wl.heads,
                    "head_dim": wl.dim, "budget": {"generated": wl.generated, "reference": wl.reference},

@@ -228,6 +228,28 @@ int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* 
                     const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
                     const int32_t* heads, void* stream);
 
+/* INT8 Q/K variant. The pages' own kernel computes Q K^T in INT8 (a SageAttention-derived kernel;
+ * veda_core.py and the Vflash guide) but does not print its quantisation recipe; this library's reading
+ * is the symmetric per-tile one: per (head, 128-row tile) scale = amax(|x|) over the tile's real rows / 127
+ * (1 when 0), stored as fp32; each code is x / scale rounded to the nearest integer, ties to even, within
+ * +-127 (padding rows stay 0). S = Q K^T runs as an s8 x s8 tensor-core product with exact int32
+ * accumulation and is multiplied by scale_q(query tile) * scale_k(key tile) * D^-0.5; P and V stay bf16.
+ * Selection is not affected (it pools the bf16 Q and K).
+ *
+ * veda_gather_int8: veda_gather with the tile written as int8 codes and its scale (arguments as
+ *   veda_gather_fp8; codes are int8 bytes [n_heads, N, D]). D must be 64 or 128.
+ * veda_quantize_int8: the same codes from tile-ordered bf16 (arguments as veda_quantize_fp8).
+ * veda_attend_int8: veda_attend on int8 codes and scales (arguments as veda_attend_fp8). D must be 128. */
+int veda_gather_int8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                     int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales, float* feats,
+                     void* stream);
+int veda_quantize_int8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim, void* codes,
+                       float* scales, void* stream);
+int veda_attend_int8(const veda_layout* layout, const void* q_codes, const void* k_codes, const float* scales_q,
+                     const float* scales_k, const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
+                     const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
+                     const int32_t* heads, void* stream);
+
 /* Synchronizes `stream`, then reads and clears this device's latched kernel error word.
  * Returns VEDA_OK, VEDA_ERR_TIMEOUT, VEDA_ERR_BAD_LIST or VEDA_ERR_CUDA. */
 int veda_sync_status(void* stream);

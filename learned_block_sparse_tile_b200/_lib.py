@@ -22,6 +22,7 @@ EXPORTS = [
     "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_score_noalloc", "veda_select", "veda_attend",
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
     "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
+    "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8",
 ]
 
 
@@ -82,7 +83,10 @@ def lib():
         L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_quantize_fp8.argtypes = [vp, p, i32, i32, p, p, vp]
         L.veda_gather_fp8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
+        L.veda_quantize_int8.argtypes = [vp, p, i32, i32, p, p, vp]
+        L.veda_gather_int8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
         L.veda_attend_fp8.argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
+        L.veda_attend_int8.argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_sync_status.argtypes = [vp]
         L.veda_last_error.restype = C.c_char_p
         L.veda_set_wait_timeout_ns.argtypes = [C.c_uint64]
@@ -225,6 +229,25 @@ def veda_attend_fp8(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx,
     _check(lib().veda_attend_fp8(layout.handle, _ptr(q_codes), _ptr(k_codes), _ptr(scales_q), _ptr(scales_k),
                                  _ptr(v_t), v_t.shape[0], v_t.shape[2], _ptr(kept_idx), _ptr(kept_cnt), _ptr(out),
                                  _strides(out), out.shape[1], _ptr(heads), _stream(stream)))
+
+
+def veda_gather_int8(layout, x, heads, codes, scales, feats=None, stream=None):
+    """veda_gather_fp8 with int8 codes (int8 or uint8 [n, N, D])."""
+    _check(lib().veda_gather_int8(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
+                                  heads.numel(), _ptr(codes), _ptr(scales), _ptr(feats), _stream(stream)))
+
+
+def veda_quantize_int8(layout, x_t, codes, scales, stream=None):
+    """x_t: bf16 [n, N, D]; codes: int8 [n, N, D]; scales: fp32 [n, n_tiles]."""
+    _check(lib().veda_quantize_int8(layout.handle, _ptr(x_t), x_t.shape[0], x_t.shape[2], _ptr(codes), _ptr(scales),
+                                    _stream(stream)))
+
+
+def veda_attend_int8(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx, kept_cnt, out, heads, stream=None):
+    """veda_attend with int8 Q/K codes ([n, N, D]) and their per-tile scales."""
+    _check(lib().veda_attend_int8(layout.handle, _ptr(q_codes), _ptr(k_codes), _ptr(scales_q), _ptr(scales_k),
+                                  _ptr(v_t), v_t.shape[0], v_t.shape[2], _ptr(kept_idx), _ptr(kept_cnt), _ptr(out),
+                                  _strides(out), out.shape[1], _ptr(heads), _stream(stream)))
 
 
 def veda_sync_status(stream=None):

@@ -71,11 +71,15 @@ struct AttendArgs {
     const float* scales_k;
 };
 
-// kFp8: Q and K are e4m3 codes with per-tile scales (S = Q K^T on the kind::f8f6f4 path); V stays bf16.
-template <int D, bool kFp8 = false>
+// Q/K formats: bf16, or 8-bit codes with per-tile scales: e4m3 (S = Q K^T on the kind::f8f6f4 path) or
+// int8 (kind::i8, S in int32). V stays bf16 in every format.
+enum QKFormat : int { kQKBf16 = 0, kQKE4M3 = 1, kQKI8 = 2 };
+
+template <int D, int kQK = kQKBf16>
 struct AttendCfg {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-    static_assert(!kFp8 || D == 128, "the FP8 Q/K variant is built for head_dim 128");
+    static constexpr bool kFp8 = kQK != kQKBf16;  // Q and K are 8-bit codes (1 byte per element)
+    static_assert(!kFp8 || D == 128, "the 8-bit Q/K variants are built for head_dim 128");
     static constexpr int kWarps = 12;
     static constexpr int kThreads = 32 * kWarps;
     static constexpr int kQKBytes = 128 * D * (kFp8 ? 1 : 2);  // one Q or K tile
@@ -94,7 +98,9 @@ struct AttendCfg {
     static constexpr int kOffV = kOffK + kKStages * kQKBytes;
     static constexpr int kSmem = kOffV + kVStages * kTileBytes;
     static constexpr uint32_t kTmemCols = 512;  // S/P of group 0, S/P of group 1, O of group 0, O of group 1
-    static constexpr uint32_t kIdescS = kFp8 ? ptx::idesc_e4m3_f32(128, 128) : ptx::idesc_bf16_f32(128, 128, false, false);
+    static constexpr uint32_t kIdescS = kQK == kQKI8    ? ptx::idesc_s8_s32(128, 128)
+                                        : kQK == kQKE4M3 ? ptx::idesc_e4m3_f32(128, 128)
+                                                         : ptx::idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, false, true);
 };
 
@@ -161,11 +167,12 @@ __device__ __forceinline__ void decode_item(const AttendArgs& a, int item, int* 
 // Tiles of an item that softmax group w handles: the item-local tiles j = w, w + 2, ...
 __device__ __forceinline__ int group_tiles(int n, int w) { return (n - w + 1) >> 1; }
 
-template <int D, bool kFp8>
+template <int D, int kQK>
 __global__ void __launch_bounds__(384, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const AttendArgs a) {
-    using C = AttendCfg<D, kFp8>;
+    using C = AttendCfg<D, kQK>;
+    constexpr bool kFp8 = C::kFp8;  // 8-bit Q/K codes (either format)
     constexpr int KS = C::kKStages, VS = C::kVStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw;
@@ -319,11 +326,16 @@ __global__ void __launch_bounds__(384, 1)
                         ptx::tc_fence_after();
                         const uint64_t dks = dk + uint64_t(ks * (C::kQKBytes >> 4));
                         if constexpr (kFp8) {
-                            // e4m3: a 128-byte row holds all 128 dims; K = 32 per MMA (32 bytes along the row)
+                            // 8-bit codes: a 128-byte row holds all 128 dims; K = 32 per MMA (32 bytes along the row)
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                ptx::mma_f8_ss_w(tmem + 128 * w, dq + uint64_t(kk * 2), dks + uint64_t(kk * 2), C::kIdescS,
-                                                 kk > 0);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                if constexpr (kQK == kQKI8)
+                                    ptx::mma_i8_ss_w(tmem + 128 * w, dq + uint64_t(kk * 2), dks + uint64_t(kk * 2), C::kIdescS,
+                                                     kk > 0);
+                                else
+                                    ptx::mma_f8_ss_w(tmem + 128 * w, dq + uint64_t(kk * 2), dks + uint64_t(kk * 2), C::kIdescS,
+                                                     kk > 0);
+                            }
                         } else {
                             // K = 16 per MMA: 32 bytes along a 128-byte row, then the next 64-column box (16 KB on)
 #pragma unroll
@@ -415,6 +427,19 @@ __global__ void __launch_bounds__(384, 1)
                 for (int i = 0; i < 4; ++i)
                     ptx::tmem_ld32(t_s + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(s + 32 * i));
                 ptx::tmem_wait_ld();
+                if constexpr (kQK == kQKI8) {
+                    // int32 -> fp32, exactly: adding the bit pattern of 1.5 * 2^23 puts |S| < 2^22 in the
+                    // low mantissa bits of a float in [2^23, 2^24); subtracting 1.5 * 2^23 is then exact
+                    const uint64_t magic = ptx::f2_pack(-12582912.f, -12582912.f);
+#pragma unroll
+                    for (int c = 0; c < 128; c += 2) {
+                        float f0, f1;
+                        ptx::f2_unpack(ptx::f2_add(ptx::f2_pack(__uint_as_float(s[c] + 0x4B400000u),
+                                                                __uint_as_float(s[c + 1] + 0x4B400000u)), magic), f0, f1);
+                        s[c] = __float_as_uint(f0);
+                        s[c + 1] = __float_as_uint(f1);
+                    }
+                }
                 if (vc < 128) {
 #pragma unroll
                     for (int c = 0; c < 128; ++c)

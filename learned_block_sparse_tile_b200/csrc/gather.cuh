@@ -6,8 +6,8 @@
 // One CTA per (tile, head): 256 threads move the tile's 128 rows of D bf16 with 16-byte loads (each
 // row is one contiguous 2*D-byte run of the source), keep them in registers, write them to the
 // head-major tile-ordered output and reduce them column-wise in the same pass. HBM bound.
-// The kCodes form writes the tile as e4m3 codes with its per-tile scale (the FP8 Q/K variant's
-// quantisation, quant.cuh) instead of bf16, from the same registers.
+// kCode != 0 writes the tile as 8-bit codes (e4m3 or int8) with its per-tile scale (the 8-bit Q/K
+// variants' quantisation, quant.cuh) instead of bf16, from the same registers.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,8 +25,8 @@ struct GatherArgs {
     const int32_t* perm;          // [n_slots]
     const int32_t* valid_count;   // [n_tiles]
     __nv_bfloat16* x_t;           // [n_heads, n_slots, D] (bf16 form)
-    uint8_t* codes;               // [n_heads, n_slots, D] e4m3 (kCodes form)
-    float* scales;                // [n_heads, n_tiles] (kCodes form)
+    uint8_t* codes;               // [n_heads, n_slots, D] 8-bit codes (kCode != 0)
+    float* scales;                // [n_heads, n_tiles] (kCode != 0)
     int32_t n_tiles;
     float* feats;                 // [n_heads, n_video, 3D] or null
     int64_t n_slots;
@@ -35,7 +35,7 @@ struct GatherArgs {
     int* err;                     // latched error bits; bit 4 = head index out of range
 };
 
-template <int D, bool kCodes = false>
+template <int D, int kCode = 0>
 __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
     constexpr int kTpr = D / 8;          // threads per row (8 bf16 = 16 bytes each)
     constexpr int kRpp = 256 / kTpr;     // rows per pass
@@ -61,9 +61,9 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
         v[p] = pr >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + int64_t(pr) * a.s0)) : make_uint4(0, 0, 0, 0);
     }
     const int64_t base = (int64_t(hh) * a.n_slots + int64_t(tile) * 128) * D + c * 8;
-    if constexpr (kCodes) {
+    if constexpr (kCode != 0) {
         __shared__ float red8[8];
-        quantize_tile<D>(v, r0, vc, red8, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
+        quantize_tile<D, kCode>(v, r0, vc, red8, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
     } else {
         __nv_bfloat16* dst = a.x_t + base;
 #pragma unroll

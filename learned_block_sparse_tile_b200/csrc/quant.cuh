@@ -1,8 +1,10 @@
-// Per-tile FP8 (e4m3) quantisation of tile-ordered Q or K for the FP8 attention variant.
-// Not on the pages (their kernel quantises to INT8 by an unpublished recipe). Reading adopted: for each
-// (head, 128-row tile) the scale is s = amax(|x|) over the tile's real rows / 448 (1 when that is 0), kept
-// as fp32; each code is x / s rounded to nearest-even e4m3 with saturation at +-448. Padding rows
-// are zero and stay zero. HBM bound: reads 2 bytes and writes 1 byte per element.
+// Per-tile quantisation of tile-ordered Q or K for the 8-bit attention variants.
+// The pages' own kernel computes Q K^T in INT8 by a recipe they do not print. Readings adopted, per
+// (head, 128-row tile), with the scale kept as fp32 (1 when the amax is 0):
+//  e4m3: s = amax(|x| over the tile's real rows) / 448; code = x / s rounded to nearest-even e4m3,
+//        saturating at +-448;
+//  int8: s = amax / 127; code = x / s rounded to the nearest integer, ties to even, within +-127.
+// Padding rows are zero and stay zero. HBM bound in principle: reads 2 bytes and writes 1 byte per element.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -48,12 +50,22 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Code formats of the 8-bit variants.
+enum TileCode : int { kCodeE4M3 = 1, kCodeI8 = 2 };
+
+// Round-to-odd quotient to an int8 code: nearest integer, ties to even (the fp32 round-to-odd value
+// carries enough bits for that rounding to equal rounding the exact quotient), within +-127.
+__device__ __forceinline__ uint32_t i8_code(float q_odd) {
+    const int c = __float2int_rn(q_odd);
+    return uint32_t(max(-127, min(127, c))) & 0xFFu;
+}
+
 // Quantises one (head, 128-row tile) held by a 256-thread CTA: D / 8 threads cover a row (8 bf16 = 16
 // bytes each), thread tid holds rows r0 + p * kRpp (r0 = tid / (D / 8)) of its 8 columns in v[p]. Rows
 // from vc on are padding (zero, and left out of the amax). Writes the tile's scale (thread 0) and the
 // codes of all 128 rows to codes (this thread's column chunk of row 0; rows are D bytes apart). Contains a
 // block barrier: every thread of the CTA must call it.
-template <int D>
+template <int D, int kCode>
 __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, float* red8, uint8_t* codes,
                                               float* scale) {
     constexpr int kTpr = D / 8;
@@ -78,7 +90,7 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
     float m = red8[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) m = fmaxf(m, red8[w]);
-    const float s = m > 0.f ? m / 448.f : 1.f;
+    const float s = m > 0.f ? m / (kCode == kCodeI8 ? 127.f : 448.f) : 1.f;
     const float inv = 1.f / s;
     if (threadIdx.x == 0) *scale = s;
 #pragma unroll
@@ -88,8 +100,12 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
-            w[e] = uint32_t(e4m3x2(quotient_round_odd(f0.x, s, inv), quotient_round_odd(f0.y, s, inv))) |
-                   (uint32_t(e4m3x2(quotient_round_odd(f1.x, s, inv), quotient_round_odd(f1.y, s, inv))) << 16);
+            const float q0 = quotient_round_odd(f0.x, s, inv), q1 = quotient_round_odd(f0.y, s, inv);
+            const float q2 = quotient_round_odd(f1.x, s, inv), q3 = quotient_round_odd(f1.y, s, inv);
+            if constexpr (kCode == kCodeI8)
+                w[e] = i8_code(q0) | (i8_code(q1) << 8) | (i8_code(q2) << 16) | (i8_code(q3) << 24);
+            else
+                w[e] = uint32_t(e4m3x2(q0, q1)) | (uint32_t(e4m3x2(q2, q3)) << 16);
         }
         *reinterpret_cast<uint2*>(codes + int64_t(r0 + p * kRpp) * D) = make_uint2(w[0], w[1]);
     }
@@ -97,8 +113,8 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
 
 // One CTA per (tile, head), 256 threads, over a tile-ordered bf16 tensor. HBM bound: reads 2 bytes and
 // writes 1 byte per element.
-template <int D>
-__global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
+template <int D, int kCode>
+__global__ void __launch_bounds__(256) quantize_kernel(const QuantArgs a) {
     constexpr int kTpr = D / 8;
     constexpr int kRpp = 256 / kTpr;
     constexpr int kPasses = 128 / kRpp;
@@ -110,7 +126,7 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
     uint4 v[kPasses];
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) v[p] = *reinterpret_cast<const uint4*>(a.x_t + base + int64_t(r0 + p * kRpp) * D);
-    quantize_tile<D>(v, r0, vc, red, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
+    quantize_tile<D, kCode>(v, r0, vc, red, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
 }
 
 }  // namespace veda

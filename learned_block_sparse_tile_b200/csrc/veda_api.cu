@@ -34,7 +34,7 @@ struct DeviceState {
     bool init = false;
     int sms = 0;
     int* err = nullptr;  // device address of g_err
-    bool attend_attr[4] = {false, false, false, false};
+    bool attend_attr[6] = {false, false, false, false, false, false};  // (head_dim 128) + 2 * Q/K format
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -219,16 +219,17 @@ extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64
     return launch_check("gather_pool_kernel");
 }
 
-extern "C" int veda_gather_fp8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
-                               int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales,
-                               float* feats, void* stream) {
+// veda_gather_fp8 / veda_gather_int8: the gather writing 8-bit codes and per-tile scales.
+static int gather_codes(const char* who, int code, const veda_layout* layout, const void* x,
+                        const int64_t x_strides[3], int32_t h_total, int32_t dim, const int32_t* heads, int32_t n_heads,
+                        void* codes, float* scales, float* feats, void* stream) {
     clear_error();
-    if (!layout || !x || !heads || !codes || !scales) return fail(VEDA_ERR_INVALID, "veda_gather_fp8: NULL argument");
-    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_gather_fp8: head_dim must be 64 or 128");
-    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_gather_fp8: head counts must be positive");
-    if (int rc = check_strided(x_strides, x, "veda_gather_fp8 x")) return rc;
+    if (!layout || !x || !heads || !codes || !scales) return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, std::string(who) + ": head_dim must be 64 or 128");
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, std::string(who) + ": head counts must be positive");
+    if (int rc = check_strided(x_strides, x, who)) return rc;
     if (!aligned16(codes) || !aligned16(scales) || (feats && !aligned16(feats)))
-        return fail(VEDA_ERR_INVALID, "veda_gather_fp8: outputs need 16-byte alignment");
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": outputs need 16-byte alignment");
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
     const DeviceCopy* dc;
@@ -252,11 +253,32 @@ extern "C" int veda_gather_fp8(const veda_layout* layout, const void* x, const i
     a.err = ds->err;
     dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dim == 128)
-        gather_pool_kernel<128, true><<<grid, 256, 0, s>>>(a);
-    else
-        gather_pool_kernel<64, true><<<grid, 256, 0, s>>>(a);
-    return launch_check("gather_pool_kernel (e4m3 codes)");
+    if (code == kCodeI8) {
+        if (dim == 128)
+            gather_pool_kernel<128, kCodeI8><<<grid, 256, 0, s>>>(a);
+        else
+            gather_pool_kernel<64, kCodeI8><<<grid, 256, 0, s>>>(a);
+    } else {
+        if (dim == 128)
+            gather_pool_kernel<128, kCodeE4M3><<<grid, 256, 0, s>>>(a);
+        else
+            gather_pool_kernel<64, kCodeE4M3><<<grid, 256, 0, s>>>(a);
+    }
+    return launch_check("gather_pool_kernel (8-bit codes)");
+}
+
+extern "C" int veda_gather_fp8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                               int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales,
+                               float* feats, void* stream) {
+    return gather_codes("veda_gather_fp8", kCodeE4M3, layout, x, x_strides, h_total, dim, heads, n_heads, codes,
+                        scales, feats, stream);
+}
+
+extern "C" int veda_gather_int8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                                int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales,
+                                float* feats, void* stream) {
+    return gather_codes("veda_gather_int8", kCodeI8, layout, x, x_strides, h_total, dim, heads, n_heads, codes,
+                        scales, feats, stream);
 }
 
 extern "C" size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim) {
@@ -364,26 +386,27 @@ extern "C" int veda_select(const veda_layout* layout, const float* scores, int32
     return launch_check("select_kernel");
 }
 
-template <int D, bool kFp8>
+template <int D, int kQK>
 static int launch_attend(DeviceState* ds, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttendArgs& a, cudaStream_t s) {
-    using C = AttendCfg<D, kFp8>;
-    const int slot = (D == 128) + 2 * kFp8;
+    using C = AttendCfg<D, kQK>;
+    const int slot = (D == 128) + 2 * kQK;
     if (!ds->attend_attr[slot]) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
         ds->attend_attr[slot] = true;
     }
     const int grid = std::max(1, std::min(a.n_items, ds->sms));
-    attend_kernel<D, kFp8><<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, a);
+    attend_kernel<D, kQK><<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, a);
     return launch_check("attend_kernel");
 }
 
 static int attend_common(const veda_layout* layout, const void* q, const void* k, const float* sq, const float* sk,
                          const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
                          const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
-                         const int32_t* heads, void* stream, bool fp8) {
-    const char* who = fp8 ? "veda_attend_fp8" : "veda_attend";
+                         const int32_t* heads, void* stream, int qk) {
+    const bool fp8 = qk != kQKBf16;  // 8-bit Q/K codes (e4m3 or int8)
+    const char* who = qk == kQKI8 ? "veda_attend_int8" : fp8 ? "veda_attend_fp8" : "veda_attend";
     if (!layout || !q || !k || !v_t || !kept_idx || !kept_cnt || !out || !heads || (fp8 && (!sq || !sk)))
         return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
     if (fp8 ? dim != 128 : (dim != 64 && dim != 128))
@@ -431,8 +454,9 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
     a.scales_q = sq;
     a.scales_k = sk;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (fp8) return launch_attend<128, true>(ds, mq, mk, mv, a, s);
-    return dim == 128 ? launch_attend<128, false>(ds, mq, mk, mv, a, s) : launch_attend<64, false>(ds, mq, mk, mv, a, s);
+    if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, mq, mk, mv, a, s);
+    if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, mq, mk, mv, a, s);
+    return dim == 128 ? launch_attend<128, kQKBf16>(ds, mq, mk, mv, a, s) : launch_attend<64, kQKBf16>(ds, mq, mk, mv, a, s);
 }
 
 extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
@@ -440,7 +464,7 @@ extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const voi
                            const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
     clear_error();
     return attend_common(layout, q_t, k_t, nullptr, nullptr, v_t, n_heads, dim, kept_idx, kept_cnt, out, out_strides,
-                         h_total, heads, stream, false);
+                         h_total, heads, stream, kQKBf16);
 }
 
 extern "C" int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* k_codes,
@@ -449,17 +473,26 @@ extern "C" int veda_attend_fp8(const veda_layout* layout, const void* q_codes, c
                                const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
     clear_error();
     return attend_common(layout, q_codes, k_codes, scales_q, scales_k, v_t, n_heads, dim, kept_idx, kept_cnt, out,
-                         out_strides, h_total, heads, stream, true);
+                         out_strides, h_total, heads, stream, kQKE4M3);
 }
 
-extern "C" int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim,
-                                 void* codes, float* scales, void* stream) {
+extern "C" int veda_attend_int8(const veda_layout* layout, const void* q_codes, const void* k_codes,
+                                const float* scales_q, const float* scales_k, const void* v_t, int32_t n_heads,
+                                int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                                const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
     clear_error();
-    if (!layout || !x_t || !codes || !scales) return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: NULL argument");
-    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: head_dim must be 64 or 128");
-    if (n_heads <= 0) return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: n_heads must be positive");
+    return attend_common(layout, q_codes, k_codes, scales_q, scales_k, v_t, n_heads, dim, kept_idx, kept_cnt, out,
+                         out_strides, h_total, heads, stream, kQKI8);
+}
+
+static int quantize_codes(const char* who, int code, const veda_layout* layout, const void* x_t, int32_t n_heads,
+                          int32_t dim, void* codes, float* scales, void* stream) {
+    clear_error();
+    if (!layout || !x_t || !codes || !scales) return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, std::string(who) + ": head_dim must be 64 or 128");
+    if (n_heads <= 0) return fail(VEDA_ERR_INVALID, std::string(who) + ": n_heads must be positive");
     if (!aligned16(x_t) || !aligned16(codes) || !aligned16(scales))
-        return fail(VEDA_ERR_INVALID, "veda_quantize_fp8: buffers need 16-byte alignment");
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": buffers need 16-byte alignment");
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
     const DeviceCopy* dc;
@@ -473,11 +506,28 @@ extern "C" int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int
     a.n_tiles = layout->desc.n_tiles;
     dim3 grid(unsigned(layout->desc.n_tiles), unsigned(n_heads));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dim == 128)
-        quantize_fp8_kernel<128><<<grid, 256, 0, s>>>(a);
-    else
-        quantize_fp8_kernel<64><<<grid, 256, 0, s>>>(a);
-    return launch_check("quantize_fp8_kernel");
+    if (code == kCodeI8) {
+        if (dim == 128)
+            quantize_kernel<128, kCodeI8><<<grid, 256, 0, s>>>(a);
+        else
+            quantize_kernel<64, kCodeI8><<<grid, 256, 0, s>>>(a);
+    } else {
+        if (dim == 128)
+            quantize_kernel<128, kCodeE4M3><<<grid, 256, 0, s>>>(a);
+        else
+            quantize_kernel<64, kCodeE4M3><<<grid, 256, 0, s>>>(a);
+    }
+    return launch_check("quantize_kernel");
+}
+
+extern "C" int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim,
+                                 void* codes, float* scales, void* stream) {
+    return quantize_codes("veda_quantize_fp8", kCodeE4M3, layout, x_t, n_heads, dim, codes, scales, stream);
+}
+
+extern "C" int veda_quantize_int8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim,
+                                  void* codes, float* scales, void* stream) {
+    return quantize_codes("veda_quantize_int8", kCodeI8, layout, x_t, n_heads, dim, codes, scales, stream);
 }
 
 extern "C" int veda_sync_status(void* stream) {

@@ -25,9 +25,12 @@ class VedaLayer:
 
     LAUNCHES_PER_GROUP = 8  # gather q, gather k, 3 score GEMMs, select, gather v, attend
 
-    def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False):
+    def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False,
+                 int8_qk=False):
         self.seq_len, self.heads, self.dim = int(seq_len), int(heads), int(dim)
-        self.fp8_qk = bool(fp8_qk)
+        if fp8_qk and int8_qk:
+            raise ValueError("VedaLayer: choose one of fp8_qk and int8_qk")
+        self.fp8_qk, self.int8_qk = bool(fp8_qk), bool(int8_qk)
         self.device = torch.device(device)
         lps = L.veda_least_padding_box(target[1])
         groups = {}
@@ -50,9 +53,10 @@ class VedaLayer:
                      scores=torch.empty(n, lay.n_video, lay.n_video, dtype=torch.float32, device=dev),
                      kept_idx=torch.empty(n, lay.n_video, lay.max_kept, dtype=torch.int32, device=dev),
                      kept_cnt=torch.empty(n, lay.n_video, dtype=torch.int32, device=dev))
-            if self.fp8_qk:  # Q and K are gathered straight to e4m3 codes with per-tile scales
-                g.update(q8=torch.empty(n, lay.n_slots, dim, dtype=torch.uint8, device=dev),
-                         k8=torch.empty(n, lay.n_slots, dim, dtype=torch.uint8, device=dev),
+            if self.fp8_qk or self.int8_qk:  # Q and K are gathered straight to 8-bit codes with per-tile scales
+                code_t = torch.int8 if self.int8_qk else torch.uint8
+                g.update(q8=torch.empty(n, lay.n_slots, dim, dtype=code_t, device=dev),
+                         k8=torch.empty(n, lay.n_slots, dim, dtype=code_t, device=dev),
                          sq=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev),
                          sk=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev))
             else:
@@ -114,9 +118,10 @@ class VedaLayer:
         for g in self.groups:
             lay = g["layout"]
             m = mark("gather_qk")
-            if self.fp8_qk:
-                L.veda_gather_fp8(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st)
-                L.veda_gather_fp8(lay, k, g["heads"], g["k8"], g["sk"], g["feats_k"], st)
+            if self.fp8_qk or self.int8_qk:
+                gather = L.veda_gather_int8 if self.int8_qk else L.veda_gather_fp8
+                gather(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st)
+                gather(lay, k, g["heads"], g["k8"], g["sk"], g["feats_k"], st)
             else:
                 L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st)
                 L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st)
@@ -130,10 +135,10 @@ class VedaLayer:
             m = mark("gather_v")
             L.veda_gather(lay, v, g["heads"], g["v_t"], None, st)
             done(m)
-            if self.fp8_qk:
+            if self.fp8_qk or self.int8_qk:
                 m = mark("attend")
-                L.veda_attend_fp8(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"],
-                                  out, g["heads"], st)
+                attend = L.veda_attend_int8 if self.int8_qk else L.veda_attend_fp8
+                attend(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
                 done(m)
             else:
                 m = mark("attend")

@@ -40,12 +40,12 @@ def built():
 
 
 @pytest.mark.parametrize("name", ["single", "mixed", "long", "sweep_tiles24", "sweep_r025", "sweep_r050",
-                                  "sweep_dense", "sweep_fp8"])
+                                  "sweep_dense", "sweep_fp8", "sweep_int8"])
 def test_full_size_layer(name):
     wl = V.workload(name)
     x = inputs(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk)
+                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk)
     layer.set_projections(x["pq"], x["pk"])
     out = torch.full_like(x["dq"], 7.0)
     layer.forward(x["dq"], x["dk"], x["dv"], out)
@@ -90,12 +90,12 @@ def test_full_size_layer(name):
         q_tiles = V.sample_tiles(lay_o.n_tiles, lay_o.n_video, 3, seed=int(rng.integers(1 << 30)))
         qt, kt, vt = (O.gather(a, lay_o, heads) for a in (x["nq"], x["nk"], x["nv"]))
         lists = lambda hh, i: np.flatnonzero(mask[hh, i])
-        attend = O.attend_tiles_fp8 if wl.fp8_qk else O.attend_tiles
+        attend = O.attend_tiles_fp8 if wl.fp8_qk else O.attend_tiles_int8 if wl.int8_qk else O.attend_tiles
         o_t = attend(qt, kt, vt, lay_o, lists, q_tiles=q_tiles)
         err = _sampled_error(got_out, o_t, lay_o, heads, q_tiles)
         assert err.max() <= ATT_MAX_ABS and err.mean() <= ATT_MEAN_ABS, (err.max(), err.mean())
-        if wl.fp8_qk:
-            # against unquantised attention: no worse than the FP8 reading's own quantisation error
+        if wl.fp8_qk or wl.int8_qk:
+            # against unquantised attention: no worse than the 8-bit reading's own quantisation error
             o_ref = O.attend_tiles(qt, kt, vt, lay_o, lists, q_tiles=q_tiles)
             q_err = _sampled_error(o_t, o_ref, lay_o, list(range(len(heads))), q_tiles, packed=False)
             err_ref = _sampled_error(got_out, o_ref, lay_o, heads, q_tiles)

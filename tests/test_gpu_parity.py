@@ -308,3 +308,95 @@ def test_select_block_widths(width):
     assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
     _, mask = oracle_kept(lay_o, s, O.column_blocks(lay_o, gen, ref))
     compare_lists(dict(kept_idx=idx, kept_cnt=cnt), mask, lay_o)
+
+
+def test_int8_qk_variant():
+    # quantiser (standalone and fused into the gather): scales and codes equal the oracle's INT8 reading bit
+    # for bit; attention: against the oracle's INT8 reading (bf16 tolerance) and against unquantised
+    # attention (no worse than the reading's own quantisation error plus that tolerance)
+    c = case("small_d128")
+    wl = c.wl
+    q, k, v = f32(c.q), f32(c.k), f32(c.v)
+    out = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    want_i8 = np.full(out.shape, np.nan)
+    want_ref = np.full(out.shape, np.nan)
+    for box, heads in c.groups:
+        res = c.run_group(box, heads)
+        lay = res["layout"]
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        n = len(heads)
+        q8 = torch.empty(n, lay.n_slots, wl.dim, dtype=torch.int8, device="cuda")
+        k8, q8g = torch.empty_like(q8), torch.empty_like(q8)
+        sq = torch.empty(n, lay.n_tiles, dtype=torch.float32, device="cuda")
+        sk, sqg = torch.empty_like(sq), torch.empty_like(sq)
+        L.veda_quantize_int8(lay, res["q_t"], q8, sq)
+        L.veda_quantize_int8(lay, res["k_t"], k8, sk)
+        L.veda_gather_int8(lay, c.dq, res["heads"], q8g, sqg)
+        L.veda_attend_int8(lay, q8, k8, sq, sk, res["v_t"], res["kept_idx"], res["kept_cnt"], out, res["heads"])
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        assert torch.equal(q8, q8g) and torch.equal(sq, sqg)
+        qt, kt, vt = (O.gather(x, lay_o, heads) for x in (q, k, v))
+        for x_t, codes, scales in ((qt, q8, sq), (kt, k8, sk)):
+            want_codes, want_scales = O.quantize_int8_tiles(x_t, lay_o)
+            assert np.array_equal(f32(scales).astype(np.float64), want_scales)
+            assert np.array_equal(codes.cpu().numpy().astype(np.float64).transpose(1, 0, 2), want_codes)
+        _, mask = oracle_kept(lay_o, f32(res["scores"]), O.column_blocks(lay_o, wl.generated, wl.reference))
+        lists = lambda hh, i: np.flatnonzero(mask[hh, i])
+        O.scatter(want_i8, O.attend_tiles_int8(qt, kt, vt, lay_o, lists), lay_o, heads)
+        O.scatter(want_ref, O.attend_tiles(qt, kt, vt, lay_o, lists), lay_o, heads)
+    got = f32(out)
+    mx, mean = attention_error(got, want_i8)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    mx, _ = attention_error(got, want_ref)
+    q_err, _ = attention_error(want_i8, want_ref)
+    assert mx <= q_err + ATT_MAX_ABS, (mx, q_err)
+
+
+def _int8_midpoint_tile(rng, mode, D):
+    """Tile of bf16 bits whose quotients by the tile's fp32 scale sit on integer rounding midpoints. 'tie':
+    the scale is a power of two (amax = 127 2^-k) and x = (j + 1/2) 2^-k, so x / s is exactly j + 1/2.
+    'near': amax has at most 6 significant bits, so x = amax / 2 is exact in bf16 and x / (amax / 127) is
+    exactly 63.5; the fp32 rounding of the stored scale alone moves x / s off it (127 is prime, so
+    amax / 127 is never exact in fp32 for these amax)."""
+    if mode == "tie":
+        k = int(rng.integers(1, 8))
+        amax = 127.0 * 2.0 ** -k
+        xs = (np.arange(127) + 0.5) * 2.0 ** -k
+    else:
+        amax = float(rng.choice([13.0, 5.75, 27.5, 1.5, 0.8125, 19.0, 43.0, 2.75]))
+        xs = np.array([amax / 2, amax / 4, 3 * amax / 8])
+    bits = _bf16(np.concatenate([xs, -xs]))
+    tile = rng.choice(bits, size=(128, D))
+    tile[0, 0] = _bf16([amax])[0]
+    return tile
+
+
+def test_int8_codes_at_rounding_midpoints():
+    c = case("padded_tiny")
+    wl = c.wl
+    box, heads = c.groups[0]
+    lay = c.run_group(box, heads)["layout"]
+    lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+    D, N = wl.dim, lay.n_slots
+    rng = np.random.default_rng(12)
+    bits = np.zeros((N, D), dtype=np.uint16)
+    for i in range(lay.n_tiles):
+        tile = _int8_midpoint_tile(rng, "near" if i % 2 else "tie", D)
+        tile[int(lay_o.valid_count[i]):] = 0
+        bits[i * 128:(i + 1) * 128] = tile
+    x_t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(1, N, D).cuda()
+    codes = torch.empty(1, N, D, dtype=torch.int8, device="cuda")
+    scales = torch.empty(1, lay.n_tiles, dtype=torch.float32, device="cuda")
+    L.veda_quantize_int8(lay, x_t, codes, scales)
+    perm = lay_o.perm
+    real = np.flatnonzero(perm >= 0)
+    x = torch.zeros(wl.seq_len, 1, D, dtype=torch.bfloat16)
+    x[torch.from_numpy(perm[real]).long(), 0] = x_t[0].cpu()[torch.from_numpy(real).long()]
+    codes_g, scales_g = torch.empty_like(codes), torch.empty_like(scales)
+    L.veda_gather_int8(lay, x.cuda(), torch.zeros(1, dtype=torch.int32, device="cuda"), codes_g, scales_g)
+    assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+    want_codes, want_scales = O.quantize_int8_tiles(f32(x_t).transpose(1, 0, 2), lay_o)
+    for cd, sc in ((codes, scales), (codes_g, scales_g)):
+        assert np.array_equal(f32(sc).astype(np.float64), want_scales)
+        got = cd.cpu().numpy().astype(np.float64).transpose(1, 0, 2)
+        assert np.array_equal(got, want_codes), int((got != want_codes).sum())

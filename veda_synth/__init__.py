@@ -36,7 +36,7 @@ class Workload:
     ``ref_spans`` are ``(start, (T, H, W))``; ``target`` is ``(start, (T, H, W))``; every other row of
     the ``seq_len`` packed rows is a text/global row. ``head_shapes[h]`` is the target box of head
     ``h`` or ``None`` for the least-padding box. Budgets are ``(ratio, tiles)`` pairs with exactly one
-    set. ``fp8_qk`` asks for the FP8 e4m3 Q/K variant.
+    set. ``fp8_qk`` asks for the FP8 e4m3 Q/K variant, ``int8_qk`` for the INT8 one.
     """
     name: str
     heads: int
@@ -50,6 +50,7 @@ class Workload:
     bias: bool
     fp8_qk: bool = False
     note: str = ""
+    int8_qk: bool = False
     extra: dict = field(default_factory=dict, compare=False, hash=False)
 
 
@@ -91,6 +92,9 @@ def workloads():
     w["sweep_fp8"] = Workload("sweep_fp8", 24, 128, 104832, (), (0, _GRID_104K), (None,) * 24,
                               _ratio(0.10), _DENSE, True, fp8_qk=True,
                               note="FP8 e4m3 Q/K with per-tile fp32 scales, ratio 0.10")
+    w["sweep_int8"] = Workload("sweep_int8", 24, 128, 104832, (), (0, _GRID_104K), (None,) * 24,
+                               _ratio(0.10), _DENSE, True, int8_qk=True,
+                               note="INT8 Q/K with per-tile fp32 scales, ratio 0.10")
     # the 104k-token layer with 4 heads: a profiling case that still exceeds L2 (322 MB of Q/K/V)
     w["single_h4"] = Workload("single_h4", 4, 128, 104832, (), (0, _GRID_104K), (None,) * 4,
                               _ratio(0.10), _DENSE, True, note="grid (26,48,84), 4 heads, ratio 0.10 (profiling)")

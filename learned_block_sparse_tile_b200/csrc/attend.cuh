@@ -219,7 +219,16 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = a.timeout_ns;
 
-    if (warp == 0 || warp == 2) {
+    // registers: the copy/MMA warpgroup (warps 0-3) hands most of its share to the two softmax warpgroups,
+    // whose 128-column rows of S then fit without spilling. Each role sets its budget at the top of its
+    // own branch (the compiler allocates each branch within it); the budgets add up to exactly the
+    // 384 x 168 registers the block is launched with, so the increases can always be granted.
+    constexpr uint32_t kRegsLow = 56, kRegsHigh = 224;
+    static_assert(128 * kRegsLow + 256 * kRegsHigh == 384 * 168, "register split");
+    if (warp == 3) {
+        ptx::regs_dec<kRegsLow>();  // idle, but part of the copy/MMA warpgroup
+    } else if (warp == 0 || warp == 2) {
+        ptx::regs_dec<kRegsLow>();
         // ------------------------------------------------------------- producers: warp 0 Q and K, warp 2 V
         const bool kq = warp == 0;
         const int S = kq ? KS : VS;
@@ -277,6 +286,7 @@ __global__ void __launch_bounds__(384, 1)
             if (kq && issued_q > 0) ptx::mbar_wait(&B.q_full, (issued_q - 1) & 1, &never, kDrainNs);
         }
     } else if (warp == 1) {
+        ptx::regs_dec<kRegsLow>();
         // ------------------------------------------------------------- MMA issuer (whole warp, one lane issues)
         // Per item: S_0 and S_1, then for each tile j: O_(j%2) += P_j V_j, then S_(j+2). S_j lands in S
         // buffer j%2, which softmax group j%2 turns into P_j in place.
@@ -363,6 +373,7 @@ __global__ void __launch_bounds__(384, 1)
             ptx::mbar_wait(&B.drain, 0, &never, kDrainNs);
         }
     } else if (warp >= 4) {
+        ptx::regs_inc<kRegsHigh>();
         // ------------------------------------------------------------- softmax groups (warps 4-7, 8-11)
         const int w = (warp - 4) >> 2;  // group: item-local tiles j with j % 2 == w
         const int q4 = warp & 3;        // TMEM lane quarter this warp may access

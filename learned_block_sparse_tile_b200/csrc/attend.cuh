@@ -40,8 +40,9 @@
 namespace veda {
 
 // Of every 8 column pairs of a row, this many take exp2 on the FMA pipe (polynomial) and the rest on the
-// MUFU: 128 MUFU exp2 per row would cost 1024 cycles of one SMSP's MUFU per tile, more than the MMAs.
-constexpr int kPolyPairs = 3;
+// MUFU: 128 MUFU exp2 per row would cost 1024 cycles of one SMSP's MUFU per tile, more than the MMAs,
+// while each polynomial pair costs about ten issue slots. 2 measured fastest (1, 3, 4 and 5 slower).
+constexpr int kPolyPairs = 2;
 
 constexpr int kErrTimeout = 1;
 constexpr int kErrBadList = 2;

@@ -64,6 +64,7 @@ class VedaLayer:
                          k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
             self.groups.append(g)
         self.launches = self.LAUNCHES_PER_GROUP * len(self.groups)
+        self._side = torch.cuda.Stream(self.device)  # the V gathers
 
     def set_projections(self, proj_q, proj_k):
         """proj_q, proj_k: fp32 [H, 3D, D] (any device); each group keeps its heads' slices on device."""
@@ -97,27 +98,32 @@ class VedaLayer:
     def forward(self, q, k, v, out, stream=None, events=None):
         """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten.
 
-        ``events``: optional dict; CUDA event pairs recorded around each stage on ``stream`` are appended
-        under the stage names gather_qk, score, select, gather_v and attend (the page's PhaseTimer)."""
+        ``events``: optional dict; CUDA event pairs recorded around each stage are appended under the stage
+        names gather_qk, score, select, gather_v and attend (the page's PhaseTimer). gather_v runs on a
+        second stream, concurrently with score and select; the others run on ``stream``."""
         st = stream if stream is not None else torch.cuda.current_stream()
 
-        def mark(name):
+        def mark(name, on):
             if events is None:
                 return None
             e = torch.cuda.Event(enable_timing=True)
-            e.record(st)
+            e.record(on)
             events.setdefault(name, []).append([e, None])
             return name
 
-        def done(name):
+        def done(name, on):
             if name is not None:
                 e = torch.cuda.Event(enable_timing=True)
-                e.record(st)
+                e.record(on)
                 events[name][-1][1] = e
 
+        # V needs neither scores nor lists: its gather runs on a second stream while this stream scores and
+        # selects (work bound by latency and arithmetic, not by HBM); it starts after the Q/K gathers, which
+        # would otherwise share the HBM bandwidth with it, and each group's attend waits for its V
+        side = self._side
         for g in self.groups:
             lay = g["layout"]
-            m = mark("gather_qk")
+            m = mark("gather_qk", st)
             if self.fp8_qk or self.int8_qk:
                 gather = L.veda_gather_int8 if self.int8_qk else L.veda_gather_fp8
                 gather(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st)
@@ -125,23 +131,27 @@ class VedaLayer:
             else:
                 L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st)
                 L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st)
-            done(m)
-            m = mark("score")
+            done(m, st)
+            qk_done = torch.cuda.Event()
+            qk_done.record(st)
+            side.wait_event(qk_done)
+            m = mark("gather_v", side)
+            L.veda_gather(lay, v, g["heads"], g["v_t"], None, side)
+            done(m, side)
+            v_done = torch.cuda.Event()
+            v_done.record(side)
+            m = mark("score", st)
             L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"], st)
-            done(m)
-            m = mark("select")
+            done(m, st)
+            m = mark("select", st)
             L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], st)
-            done(m)
-            m = mark("gather_v")
-            L.veda_gather(lay, v, g["heads"], g["v_t"], None, st)
-            done(m)
+            done(m, st)
+            st.wait_event(v_done)
+            m = mark("attend", st)
             if self.fp8_qk or self.int8_qk:
-                m = mark("attend")
                 attend = L.veda_attend_int8 if self.int8_qk else L.veda_attend_fp8
                 attend(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
-                done(m)
             else:
-                m = mark("attend")
                 L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
-                done(m)
+            done(m, st)
         return out

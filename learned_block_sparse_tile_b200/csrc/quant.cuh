@@ -11,6 +11,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace veda {
 
 struct QuantArgs {
@@ -34,14 +36,26 @@ struct QuantArgs {
 // one FMA and rounded once, which keeps its sign and its being zero (s > 0). When |x / s| > |q| the
 // truncation is q, otherwise q one unit lower in magnitude; the inexact result is that value with its
 // last bit set. Quotients small enough to underflow round to 0 in e4m3 whatever happens here.
-__device__ __forceinline__ float quotient_round_odd(float x, float s, float inv) {
-    const float q0 = x * inv;
-    const float q = fmaf(fmaf(-q0, s, x), inv, q0);
-    const float r = fmaf(-q, s, x);
+// The last step on the bits: when x / s lies on the zero side of q (r and q of opposite signs) the
+// magnitude drops by one unit, which never borrows into the sign since |q| >= one unit.
+__device__ __forceinline__ float round_odd_bits(float q, float r) {
+    const uint32_t b = __float_as_uint(q);
     if (r == 0.f || q == 0.f) return q;
-    const uint32_t b = __float_as_uint(q), sign = b & 0x80000000u, mag = b & 0x7fffffffu;
-    const bool away = (r > 0.f) == (q > 0.f);  // the exact quotient is larger in magnitude than q
-    return __uint_as_float(sign | ((away ? mag : mag - 1u) | 1u));
+    return __uint_as_float((b - ((__float_as_uint(r) ^ b) >> 31)) | 1u);
+}
+
+// Two quotients at once on the packed f32x2 pipe; s2 = (s, s), ms2 = (-s, -s), inv2 = (1/s, 1/s).
+__device__ __forceinline__ void quotient_round_odd2(float x0, float x1, uint64_t ms2, uint64_t inv2, float& q0_odd,
+                                                    float& q1_odd) {
+    const uint64_t x = ptx::f2_pack(x0, x1);
+    const uint64_t q0 = ptx::f2_mul(x, inv2);
+    const uint64_t q = ptx::f2_fma(ptx::f2_fma(q0, ms2, x), inv2, q0);
+    const uint64_t r = ptx::f2_fma(q, ms2, x);
+    float qa, qb, ra, rb;
+    ptx::f2_unpack(q, qa, qb);
+    ptx::f2_unpack(r, ra, rb);
+    q0_odd = round_odd_bits(qa, ra);
+    q1_odd = round_odd_bits(qb, rb);
 }
 
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
@@ -92,6 +106,7 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
     for (int w = 1; w < 8; ++w) m = fmaxf(m, red8[w]);
     const float s = m > 0.f ? m / (kCode == kCodeI8 ? 127.f : 448.f) : 1.f;
     const float inv = 1.f / s;
+    const uint64_t inv2 = ptx::f2_pack(inv, inv), ms2 = ptx::f2_pack(-s, -s);
     if (threadIdx.x == 0) *scale = s;
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
@@ -100,8 +115,9 @@ __device__ __forceinline__ void quantize_tile(const uint4* v, int r0, int vc, fl
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const float2 f0 = __bfloat1622float2(h2[2 * e]), f1 = __bfloat1622float2(h2[2 * e + 1]);
-            const float q0 = quotient_round_odd(f0.x, s, inv), q1 = quotient_round_odd(f0.y, s, inv);
-            const float q2 = quotient_round_odd(f1.x, s, inv), q3 = quotient_round_odd(f1.y, s, inv);
+            float q0, q1, q2, q3;
+            quotient_round_odd2(f0.x, f0.y, ms2, inv2, q0, q1);
+            quotient_round_odd2(f1.x, f1.y, ms2, inv2, q2, q3);
             if constexpr (kCode == kCodeI8)
                 w[e] = i8_code(q0) | (i8_code(q1) << 8) | (i8_code(q2) << 16) | (i8_code(q3) << 24);
             else

@@ -165,6 +165,12 @@ __device__ __forceinline__ void decode_item(const AttendArgs& a, int item, int* 
 }
 
 
+// A softmax group index carried as a type, so that code written once for both groups sees it as a constant.
+template <int W>
+struct GroupId {
+    static constexpr int value = W;
+};
+
 // Tiles of an item that softmax group w handles: the item-local tiles j = w, w + 2, ...
 __device__ __forceinline__ int group_tiles(int n, int w) { return (n - w + 1) >> 1; }
 
@@ -294,7 +300,8 @@ __global__ void __launch_bounds__(384, 1)
         int it = 0;              // items with tiles so far
         int ks = 0, kph = 0;     // K ring slot of the next S and its phase
         int vs = 0, vph = 0;     // V ring slot of the next PV and its phase
-        int pu[2] = {0, 0};      // tiles each group has had so far (barrier phases)
+        int pu0 = 0, pu1 = 0;    // tiles each group has had so far (barrier phases); scalars, not an
+                                 // array indexed by the group, which would live in local memory
         // shared-memory descriptors of the first Q, K and V boxes; a k-step or a ring slot only moves the
         // start address, which is the descriptor's low field (address / 16, below 2^14 for any CTA address)
         const uint64_t dq = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffQ), 16, 1024);
@@ -308,16 +315,16 @@ __global__ void __launch_bounds__(384, 1)
             const int n = item_tiles(a, hh, qt, &list, &bad);
             if (n == 0) continue;
             {
-                bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_full, it & 1, abort_flag, tmo));
-                for (int j = 0; ok && j < n + 2; ++j) {
+                // one issue step: PV of tile j - 2 and S of tile j, both of group W = j % 2 (a compile-time
+                // constant, so barrier addresses and TMEM columns are immediates)
+                auto step = [&](const int j, auto wc) -> bool {
+                    constexpr int w = decltype(wc)::value;
                     if (j >= 2) {
-                        // O_w += P V for tile jj = j - 2
-                        const int jj = j - 2, w = jj & 1, idx = pu[w] + (jj >> 1);
-                        ok = ptx::mbar_wait(&B.p_full[w], idx & 1, abort_flag, tmo) &&
-                             ptx::mbar_wait(&B.v_full[vs], vph, abort_flag, tmo) &&
-                             (jj > 0 || ptx::mbar_wait(&B.o_empty, (it & 1) ^ 1, abort_flag, tmo));
-                        ok = __all_sync(0xffffffffu, ok);
-                        if (!ok) break;
+                        const int jj = j - 2, idx = (w ? pu1 : pu0) + (jj >> 1);
+                        bool ok = ptx::mbar_wait(&B.p_full[w], idx & 1, abort_flag, tmo) &&
+                                  ptx::mbar_wait(&B.v_full[vs], vph, abort_flag, tmo) &&
+                                  (jj > 0 || ptx::mbar_wait(&B.o_empty, (it & 1) ^ 1, abort_flag, tmo));
+                        if (!__all_sync(0xffffffffu, ok)) return false;
                         ptx::tc_fence_after();
                         const uint64_t dvs = dv + uint64_t(vs * (C::kTileBytes >> 4));
                         const uint32_t o = tmem + 256 + 128 * w, p = tmem + 128 * w;
@@ -330,14 +337,10 @@ __global__ void __launch_bounds__(384, 1)
                         if (++vs == VS) vs = 0, vph ^= 1;
                     }
                     if (j < n) {
-                        // S_j = Q K_j^T into S buffer j%2
-                        const int w = j & 1;
-                        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.k_full[ks], kph, abort_flag, tmo));
-                        if (!ok) break;
+                        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&B.k_full[ks], kph, abort_flag, tmo))) return false;
                         ptx::tc_fence_after();
                         const uint64_t dks = dk + uint64_t(ks * (C::kQKBytes >> 4));
                         if constexpr (kFp8) {
-                            // 8-bit codes: a 128-byte row holds all 128 dims; K = 32 per MMA (32 bytes along the row)
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 if constexpr (kQK == kQKI8)
@@ -348,21 +351,26 @@ __global__ void __launch_bounds__(384, 1)
                                                      kk > 0);
                             }
                         } else {
-                            // K = 16 per MMA: 32 bytes along a 128-byte row, then the next 64-column box (16 KB on)
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint64_t off = uint64_t((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
                                 ptx::mma_bf16_ss_w(tmem + 128 * w, dq + off, dks + off, C::kIdescS, kk > 0);
                             }
                         }
-                        ptx::mma_commit_w(&B.s_full[w]);  // the softmax group also frees the K slot on it
+                        ptx::mma_commit_w(&B.s_full[w]);
                         if (j == n - 1) ptx::mma_commit_w(&B.q_empty);
                         if (++ks == KS) ks = 0, kph ^= 1;
                     }
+                    return true;
+                };
+                bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_full, it & 1, abort_flag, tmo));
+                for (int j = 0; ok && j < n + 2; j += 2) {
+                    ok = step(j, GroupId<0>{});
+                    if (ok && j + 1 < n + 2) ok = step(j + 1, GroupId<1>{});
                 }
             }
-            pu[0] += group_tiles(n, 0);
-            pu[1] += group_tiles(n, 1);
+            pu0 += group_tiles(n, 0);
+            pu1 += group_tiles(n, 1);
             ++it;
             __syncwarp();
             if (__any_sync(0xffffffffu, *abort_flag)) break;
@@ -383,9 +391,9 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t t_s = tmem + lane_base + 128 * w;        // S / P of this group
         const uint32_t t_o = tmem + lane_base + 256 + 128 * w;  // O of this group
         const uint32_t t_o0 = tmem + lane_base + 256;
-        int cu[2] = {0, 0};  // tiles each group has had so far (barrier phases)
+        int cu = 0;          // tiles this group has had so far (barrier phases)
         int it = 0, t = 0;   // items with tiles so far; tiles so far (K ring positions)
-        int od[2] = {0, 0};  // o_done phases: one per item in which the group had a tile
+        int od_mine = 0, od_other = 0;  // o_done phases of this group and the other: one per item with a tile
         const bool releaser = (warp & 3) == 0 && lane == 0;  // one thread per group frees K slots
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
@@ -426,7 +434,7 @@ __global__ void __launch_bounds__(384, 1)
                 // log2-domain scale of this tile's logits (the FP8 path also undoes both tiles' scales)
                 const float sl2 = kFp8 ? a.scale_log2 * (sq * __shfl_sync(0xffffffffu, my_sk, k & 31)) : a.scale_log2;
                 const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
-                const int idx = cu[w] + k;
+                const int idx = cu + k;
                 ok = ptx::mbar_wait(&B.s_full[w], idx & 1, abort_flag, tmo);
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -524,12 +532,11 @@ __global__ void __launch_bounds__(384, 1)
             // (a parity wait is only meaningful within one phase).
             const int n0 = group_tiles(n, 0), n1 = group_tiles(n, 1);
             const int nmine = w ? n1 : n0, nother = w ? n0 : n1;
-            ok = (nmine == 0 || ptx::mbar_wait(&B.o_done[w], od[w] & 1, abort_flag, tmo)) &&
-                 (nother == 0 || ptx::mbar_wait(&B.o_done[w ^ 1], od[w ^ 1] & 1, abort_flag, tmo));
-            od[0] += n0 > 0;
-            od[1] += n1 > 0;
-            cu[0] += n0;
-            cu[1] += n1;
+            ok = (nmine == 0 || ptx::mbar_wait(&B.o_done[w], od_mine & 1, abort_flag, tmo)) &&
+                 (nother == 0 || ptx::mbar_wait(&B.o_done[w ^ 1], od_other & 1, abort_flag, tmo));
+            od_mine += nmine > 0;
+            od_other += nother > 0;
+            cu += nmine;
             t += n;
             if (!ok) break;
             // merge the two groups: exchange (max, sum) per row through shared memory

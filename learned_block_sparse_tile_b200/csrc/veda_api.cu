@@ -305,32 +305,7 @@ extern "C" int veda_score(const veda_layout* layout, const float* feats_q, const
     float* qh = static_cast<float*>(workspace);
     float* kh = qh + int64_t(n_heads) * nv * dim;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    for (int side = 0; side < 2; ++side) {
-        GemmArgs g;
-        g.A = side ? feats_k : feats_q;
-        g.B = side ? proj_k : proj_q;
-        g.C = side ? kh : qh;
-        g.M = nv;
-        g.N = dim;
-        g.K = 3 * dim;
-        g.sA = int64_t(nv) * 3 * dim;
-        g.sB = int64_t(3) * dim * dim;
-        g.sC = int64_t(nv) * dim;
-        g.div = 1.f;
-        gemm_f32_kernel<false><<<dim3(unsigned((dim + 63) / 64), unsigned((nv + 63) / 64), unsigned(n_heads)), 256, 0, s>>>(g);
-    }
-    GemmArgs g;
-    g.A = qh;
-    g.B = kh;
-    g.C = scores;
-    g.M = nv;
-    g.N = nv;
-    g.K = dim;
-    g.sA = int64_t(nv) * dim;
-    g.sB = int64_t(nv) * dim;
-    g.sC = int64_t(nv) * nv;
-    g.div = float(std::sqrt(double(dim)));
-    gemm_f32_kernel<true><<<dim3(unsigned((nv + 63) / 64), unsigned((nv + 63) / 64), unsigned(n_heads)), 256, 0, s>>>(g);
+    launch_score_gemms(feats_q, feats_k, proj_q, proj_k, qh, kh, scores, nv, dim, n_heads, s);
     return launch_check("gemm_f32_kernel");
 }
 

@@ -84,32 +84,9 @@ extern "C" int veda_score_noalloc(const veda_layout* layout, const float* feats_
         const int hc = std::min(chunk, n_heads - h0);
         float* qh = base;
         float* kh = base + int64_t(hc) * nv * dim;
-        for (int side = 0; side < 2; ++side) {
-            veda::GemmArgs g;
-            g.A = (side ? feats_k : feats_q) + int64_t(h0) * nv * 3 * dim;
-            g.B = (side ? proj_k : proj_q) + int64_t(h0) * 3 * dim * dim;
-            g.C = side ? kh : qh;
-            g.M = int(nv);
-            g.N = dim;
-            g.K = 3 * dim;
-            g.sA = nv * 3 * dim;
-            g.sB = int64_t(3) * dim * dim;
-            g.sC = nv * dim;
-            g.div = 1.f;
-            veda::gemm_f32_kernel<false><<<dim3(unsigned((dim + 63) / 64), unsigned((nv + 63) / 64), unsigned(hc)), 256, 0, s>>>(g);
-        }
-        veda::GemmArgs g;
-        g.A = qh;
-        g.B = kh;
-        g.C = scores + int64_t(h0) * nv * nv;
-        g.M = int(nv);
-        g.N = int(nv);
-        g.K = dim;
-        g.sA = nv * dim;
-        g.sB = nv * dim;
-        g.sC = nv * nv;
-        g.div = float(std::sqrt(double(dim)));
-        veda::gemm_f32_kernel<true><<<dim3(unsigned((nv + 63) / 64), unsigned((nv + 63) / 64), unsigned(hc)), 256, 0, s>>>(g);
+        veda::launch_score_gemms(feats_q + int64_t(h0) * nv * 3 * dim, feats_k + int64_t(h0) * nv * 3 * dim,
+                                 proj_q + int64_t(h0) * 3 * dim * dim, proj_k + int64_t(h0) * 3 * dim * dim, qh, kh,
+                                 scores + int64_t(h0) * nv * nv, int(nv), dim, hc, s);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess)

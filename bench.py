@@ -132,7 +132,7 @@ def flops_per_pair(dim):
 def stage_bytes(layer, wl):
     """Algorithmic HBM bytes per launch of each stage, summed over head groups."""
     D, S = wl.dim, wl.seq_len
-    out = {"gather_qk": 0, "score": 0, "select": 0, "gather_v": 0, "attend": 0}
+    out = {"gather_qk": 0, "pool_qk": 0, "score": 0, "select": 0, "gather_v": 0, "attend": 0}
     for g in layer.groups:
         lay, n = g["layout"], len(g["heads_list"])
         real = n * S * D * 2
@@ -141,15 +141,18 @@ def stage_bytes(layer, wl):
         # the FP8 Q/K variant writes e4m3 codes (1 byte per element) and per-tile scales instead of bf16
         eight_bit = layer.fp8_qk or layer.int8_qk
         tiles_out = slots // 2 + n * lay.n_tiles * 4 if eight_bit else slots
-        out["gather_qk"] += 2 * (real + tiles_out + feats)
-        out["gather_v"] += real + slots
+        if layer.direct:  # Q and K are read once for the pooled features; no tile-order copies
+            out["pool_qk"] += 2 * (real + feats)
+        else:
+            out["gather_qk"] += 2 * (real + tiles_out + feats)
+            out["gather_v"] += real + slots
         sc = n * lay.n_video * lay.n_video * 4
         proj = 2 * n * 3 * D * D * 4
         hat = 2 * n * lay.n_video * D * 4
         out["score"] += 2 * feats + proj + 2 * hat + sc
         kept = int(g["kept_cnt"].sum())
         out["select"] += sc + 4 * (kept + n * lay.n_video)
-        q_in = slots // 2 if eight_bit else slots
+        q_in = slots // 2 if eight_bit else real if layer.direct else slots
         out["attend"] += q_in + real + 4 * (kept + n * lay.n_video)  # Q in, O out, lists; K/V counted as L2 reuse
     return out
 
@@ -164,7 +167,9 @@ def run_veda(args, rank, world, local):
     q, k, v = V.make_qkv(wl)
     pq, pk = V.make_projections(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk)
+                      wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk,
+                      direct={"auto": None, "gathered": False, "direct": True}[args.path])
+    direct = layer.direct
     layer.set_projections(pq, pk)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     out = torch.empty_like(dq)
@@ -229,7 +234,7 @@ def run_veda(args, rank, world, local):
         gbs = sbytes[name] / (ms * 1e-3) / 1e9 if ms > 0 else None
         stages[name] = {"ms": round(ms, 4), "bytes": sbytes[name], "gb_s": round(gbs, 1) if gbs else None,
                         "hbm_frac": round(gbs / pk_["hbm"], 3) if gbs else None}
-    traffic = recorded_traffic(args.workload, wl.dim)
+    traffic = recorded_traffic(args.workload + ("/direct" if direct else ""), wl.dim)
     dense_pairs = wl.heads * (wl.seq_len / 128.0) ** 2
     res = {
         "metric": METRIC, "value": round(ms_step / world, 4), "unit": UNIT, "n_gpus": world,
@@ -240,6 +245,8 @@ def run_veda(args, rank, world, local):
         "config": {"workload": f"{wl.name}: {wl.note}", "seq_len": wl.seq_len, "heads": wl.heads,
                    "head_dim": wl.dim, "budget": {"generated": wl.generated, "reference": wl.reference},
                    "head_groups": [list(g["box"]) for g in layer.groups],
+                   "attend_path": ("gather-free: Q/K pooled in place, tiles loaded as TMA boxes of the packed tensors"
+                                   if direct else "tile-order copies of Q/K/V (gather), then attend"),
                    "parallelism": f"replicas x{world} (one layer per rank)",
                    "l2": "no flush: per-step inputs and outputs (2.6 GB at 104k tokens) exceed the 126 MB L2"},
         "kept_tile_tflops": round(achieved_tflops, 1),
@@ -278,6 +285,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="single")
+    ap.add_argument("--path", default="auto", choices=["auto", "gathered", "direct"],
+                    help="attend on tile-order copies (gathered), on the packed tensors as TMA boxes (direct), "
+                         "or the layer's choice (auto: direct where every layout has a box form)")
     ap.add_argument("--impl", default="veda", choices=["veda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)

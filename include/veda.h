@@ -111,6 +111,18 @@ typedef struct {
 int veda_plan(const veda_span* spans, int32_t n_spans, int64_t seq_len, veda_budget generated,
               veda_budget reference, veda_layout** out);
 
+/* The layout's tiles as TMA boxes of the packed tensors, the form veda_attend_direct reads (host). A span
+ * tile is the (st, sh, sw) box of its span's grid at its origin, positions in box order (t, h, w
+ * row-major) with padding left in place; a global tile is the run of 128 rows from its first row.
+ *  box_perm    [n_slots] int32: packed row of each box position, -1 where the tile has no row
+ *  tile_coord  [n_tiles * 4] int32: span tile {span, w0, h0, t0} (span = index among the tiled spans in
+ *              tile order); global tile {-1, first row, 0, 0}
+ *  tile_mask   [n_tiles * 4] int32 bit patterns: bit c % 32 of word c / 32 set iff box position c holds
+ *              a row of the tile
+ * Any pointer may be NULL. Returns VEDA_ERR_UNSUPPORTED (and copies nothing) when the gathered path is
+ * the only one for this layout: a global tile whose rows are not consecutive, or more than 4 tiled spans. */
+int veda_layout_export_direct(const veda_layout* layout, int32_t* box_perm, int32_t* tile_coord, int32_t* tile_mask);
+
 /* Sizes and budget split of a layout (host). */
 int veda_layout_info(const veda_layout* layout, veda_layout_desc* out);
 
@@ -140,6 +152,16 @@ int veda_least_padding_box(int32_t t, int32_t h, int32_t w, int32_t box_out[3]);
  * D must be 64 or 128. */
 int veda_gather(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
                 int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, void* stream);
+
+/* The pooled features of veda_gather without the tile-order copy (veda_core.py, "predictor", pool): per
+ * video tile and head [mean | max | min] over the tile's real rows, mean = fp32 sum / count, 0 for an
+ * empty tile; the same values veda_gather writes to its feats.
+ *  x      device bf16 [S, H_total, D] with element strides x_strides[3] (S, H, D).
+ *  heads  device int32 [n_heads].
+ *  feats  device fp32 [n_heads, n_video, 3D] out.
+ * D must be 64 or 128. With veda_attend_direct this is all the scoring path needs of Q and K. */
+int veda_pool(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+              int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, void* stream);
 
 /* Workspace bytes veda_score needs (projected features of Q and K): 2 * n_heads * n_video * D * 4. */
 size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim);
@@ -196,6 +218,21 @@ int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, con
                 int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt,
                 void* out, const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
                 void* stream);
+
+/* veda_attend reading the packed tensors directly, with no tile-order copies (gather-free): every tile
+ * is loaded as a TMA box of q, k and v (veda_layout_export_direct gives the boxes). Same operation as
+ * veda_attend on the same lists; the keys of a partial span tile come in box order, so its sums run in
+ * another order (within rounding of veda_attend's).
+ *  q, k, v    device bf16 [S, H_total, D] with element strides q/k/v_strides[3] (S, H, D); bases 16-byte
+ *             aligned, S and H strides multiples of 8 elements.
+ *  heads      device int32 [n_heads]: the group's heads among the H_total.
+ *  kept_idx/cnt, out, out_strides: as for veda_attend.
+ * D must be 64 or 128. VEDA_ERR_UNSUPPORTED when the layout has no box form (see
+ * veda_layout_export_direct); veda_gather + veda_attend take every layout. */
+int veda_attend_direct(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
+                       const int64_t k_strides[3], const void* v, const int64_t v_strides[3], int32_t h_total,
+                       int32_t dim, const int32_t* heads, int32_t n_heads, const int32_t* kept_idx,
+                       const int32_t* kept_cnt, void* out, const int64_t out_strides[3], void* stream);
 
 /* FP8 Q/K variant, step 1 (not on the pages: their kernel quantises to INT8 by a recipe they do not
  * print; this follows the FP8 e4m3 variant of the 104k budget sweep). Per (head, 128-row tile) of a

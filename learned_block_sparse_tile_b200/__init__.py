@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     veda_last_error, veda_layout_export, veda_layout_info, veda_least_padding_box, veda_plan, veda_score,
     veda_score_noalloc, veda_score_workspace_bytes, veda_select, veda_set_wait_timeout_ns, veda_sync_status,
     veda_quantize_fp8, veda_gather_fp8, veda_attend_fp8, veda_quantize_int8, veda_gather_int8, veda_attend_int8,
+    veda_layout_export_direct, veda_pool, veda_attend_direct,
 )
 from .layer import VedaLayer  # noqa: F401
 from .pipeline import HostPipeline  # noqa: F401

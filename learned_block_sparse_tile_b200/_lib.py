@@ -22,7 +22,8 @@ EXPORTS = [
     "veda_gather", "veda_score_workspace_bytes", "veda_score", "veda_score_noalloc", "veda_select", "veda_attend",
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
     "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
-    "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8",
+    "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8", "veda_layout_export_direct", "veda_pool",
+    "veda_attend_direct",
 ]
 
 
@@ -71,10 +72,14 @@ def lib():
         L.veda_plan.argtypes = [C.POINTER(Span), i32, i64, Budget, Budget, C.POINTER(vp)]
         L.veda_layout_info.argtypes = [vp, C.POINTER(LayoutDesc)]
         L.veda_layout_export.argtypes = [vp, p, p, p]
+        L.veda_layout_export_direct.argtypes = [vp, p, p, p]
         L.veda_layout_destroy.argtypes = [vp]
         L.veda_layout_destroy.restype = None
         L.veda_least_padding_box.argtypes = [i32, i32, i32, C.POINTER(C.c_int32)]
         L.veda_gather.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, vp]
+        L.veda_pool.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, vp]
+        L.veda_attend_direct.argtypes = [vp, p, C.POINTER(C.c_int64), p, C.POINTER(C.c_int64), p,
+                                         C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, C.POINTER(C.c_int64), vp]
         L.veda_score_workspace_bytes.argtypes = [vp, i32, i32]
         L.veda_score_workspace_bytes.restype = C.c_size_t
         L.veda_score.argtypes = [vp, p, p, i32, i32, p, p, p, C.c_size_t, p, vp]
@@ -169,6 +174,25 @@ def veda_layout_export(layout):
     return perm, vc, allowed
 
 
+def veda_layout_export_direct(layout):
+    """(box_perm [N], tile_coord [n_tiles, 4], tile_mask [n_tiles, 4]) as int32 numpy arrays: the tiles as TMA
+    boxes of the packed tensors (raises VedaError with VEDA_ERR_UNSUPPORTED when the layout has no box form)."""
+    d = layout.desc
+    box_perm = np.empty(d.n_slots, np.int32)
+    coord = np.empty((d.n_tiles, 4), np.int32)
+    mask = np.empty((d.n_tiles, 4), np.int32)
+    _check(lib().veda_layout_export_direct(layout.handle, box_perm.ctypes.data, coord.ctypes.data, mask.ctypes.data))
+    return box_perm, coord, mask
+
+
+def veda_layout_has_box_form(layout):
+    """True when veda_attend_direct can take the layout (veda_layout_export_direct with no outputs)."""
+    rc = lib().veda_layout_export_direct(layout.handle, None, None, None)
+    if rc not in (VEDA_OK, VEDA_ERR_UNSUPPORTED):
+        _check(rc)
+    return rc == VEDA_OK
+
+
 def veda_least_padding_box(grid):
     out = (C.c_int32 * 3)()
     _check(lib().veda_least_padding_box(int(grid[0]), int(grid[1]), int(grid[2]), out))
@@ -179,6 +203,13 @@ def veda_gather(layout, x, heads, x_t, feats=None, stream=None):
     """x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; x_t: bf16 [n, N, D]; feats: fp32 [n, n_video, 3D] or None."""
     _check(lib().veda_gather(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
                              heads.numel(), _ptr(x_t), _ptr(feats), _stream(stream)))
+
+
+def veda_pool(layout, x, heads, feats, stream=None):
+    """Pooled features only (no tile copy). x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; feats: fp32
+    [n, n_video, 3D]."""
+    _check(lib().veda_pool(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads), heads.numel(),
+                           _ptr(feats), _stream(stream)))
 
 
 def veda_score_workspace_bytes(layout, n_heads, dim):
@@ -209,6 +240,14 @@ def veda_attend(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, stream=No
     _check(lib().veda_attend(layout.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), q_t.shape[0], q_t.shape[2],
                              _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1], _ptr(heads),
                              _stream(stream)))
+
+
+def veda_attend_direct(layout, q, k, v, kept_idx, kept_cnt, out, heads, stream=None):
+    """veda_attend on the packed tensors (no tile-order copies). q/k/v: bf16 [S, H, D] cuda (strided ok);
+    out: bf16 [S, H, D]; heads: int32 [n] cuda."""
+    _check(lib().veda_attend_direct(layout.handle, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                    q.shape[1], q.shape[2], _ptr(heads), heads.numel(), _ptr(kept_idx),
+                                    _ptr(kept_cnt), _ptr(out), _strides(out), _stream(stream)))
 
 
 def veda_gather_fp8(layout, x, heads, codes, scales, feats=None, stream=None):

@@ -70,6 +70,23 @@ struct AttendArgs {
     int hold_q;  // test hook: the producer withholds every Q load, so every wait on Q expires
     const float* scales_q;  // FP8 variant: [n_heads, n_tiles] per-tile scales of the e4m3 Q and K codes
     const float* scales_k;
+    // gather-free variant: per tile its box origin ({span, w0, h0, t0}, or {-1, row0, 0, 0} for a global
+    // tile) and the 128-bit mask of box positions that hold one of its rows; perm is then the box-order
+    // table (packed row per box position)
+    const int4* tile_coord;
+    const uint4* tile_mask;
+    int32_t n_map_spans;  // span map sets in use (the global set is used when n_global > 0)
+};
+
+// TMA maps of one launch. The tile-ordered variant uses set 0 only (2D maps over [n_heads * N, D]). The
+// gather-free variant has one set of 5D maps per tiled span over the packed tensors viewed as
+// [T, H, W, heads, D] (box (st, sh, sw, 1, 64)) and a set of 3D maps over [rows, heads, D] for the global
+// tiles (box (128, 1, 64)), whose row extent ends after the last global row so that a partial last tile
+// reads zeros past its rows.
+constexpr int kMapSets = 5;
+constexpr int kGlobalMapSet = kMapSets - 1;
+struct AttendMaps {
+    CUtensorMap q[kMapSets], k[kMapSets], v[kMapSets];
 };
 
 // Q/K formats: bf16, or 8-bit codes with per-tile scales: e4m3 (S = Q K^T on the kind::f8f6f4 path) or
@@ -174,10 +191,9 @@ struct GroupId {
 // Tiles of an item that softmax group w handles: the item-local tiles j = w, w + 2, ...
 __device__ __forceinline__ int group_tiles(int n, int w) { return (n - w + 1) >> 1; }
 
-template <int D, int kQK>
+template <int D, int kQK, bool kDirect>
 __global__ void __launch_bounds__(384, 1)
-    attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const AttendArgs a) {
+    attend_kernel(const __grid_constant__ AttendMaps maps, const AttendArgs a) {
     using C = AttendCfg<D, kQK>;
     constexpr bool kFp8 = C::kFp8;  // 8-bit Q/K codes (either format)
     constexpr int KS = C::kKStages, VS = C::kVStages;
@@ -216,9 +232,14 @@ __global__ void __launch_bounds__(384, 1)
         ptx::fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        ptx::tma_prefetch_desc(&tm_q);
-        ptx::tma_prefetch_desc(&tm_k);
-        ptx::tma_prefetch_desc(&tm_v);
+        const int sets = kDirect ? a.n_map_spans : 1;
+        for (int i = 0; i < kMapSets; ++i) {
+            if (i < sets || (kDirect && i == kGlobalMapSet && a.n_global > 0)) {
+                ptx::tma_prefetch_desc(&maps.q[i]);
+                ptx::tma_prefetch_desc(&maps.k[i]);
+                ptx::tma_prefetch_desc(&maps.v[i]);
+            }
+        }
     }
     if (warp == 1) ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     __syncthreads();
@@ -250,22 +271,46 @@ __global__ void __launch_bounds__(384, 1)
             if (kq && bad && lane == 0) atomicOr(a.err, kErrBadList);
             if (n == 0) continue;
             const int32_t row0 = int32_t(int64_t(hh) * a.n_slots);
+            const int head = kDirect ? __ldg(a.heads + hh) : 0;  // head index in the packed tensors
             if (kq && !a.hold_q &&
                 __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo))) {
                 if (ptx::elect_one()) {
                     ptx::mbar_arrive_expect_tx(&B.q_full, C::kQKBytes);
-                    for (int x = 0; x < C::kBoxesQK; ++x)
-                        ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &tm_q, x * (kFp8 ? 128 : 64), row0 + qt * 128,
-                                         &B.q_full);
+                    if constexpr (kDirect) {
+                        const int4 tc = __ldg(a.tile_coord + qt);
+                        for (int x = 0; x < C::kBoxes; ++x) {
+                            if (tc.x >= 0)
+                                ptx::tma_load_5d_hint(smem + C::kOffQ + x * 16384, &maps.q[tc.x], x * 64, head, tc.y,
+                                                      tc.z, tc.w, &B.q_full, keep);
+                            else
+                                ptx::tma_load_3d_hint(smem + C::kOffQ + x * 16384, &maps.q[kGlobalMapSet], x * 64, head,
+                                                      tc.y, &B.q_full, keep);
+                        }
+                    } else {
+                        for (int x = 0; x < C::kBoxesQK; ++x)
+                            ptx::tma_load_2d(smem + C::kOffQ + x * 16384, &maps.q[0], x * (kFp8 ? 128 : 64),
+                                             row0 + qt * 128, &B.q_full);
+                    }
                 }
                 __syncwarp();
                 ++issued_q;
             }
             if (__any_sync(0xffffffffu, *abort_flag)) break;
             int mine = 0;
+            int4 cmine = make_int4(0, 0, 0, 0);  // gather-free variant: box origin of this lane's tile
             for (int j = 0; j < n; ++j) {
-                if ((j & 31) == 0) mine = (j + lane < n) ? __ldg(list + j + lane) : 0;
+                if ((j & 31) == 0) {
+                    mine = (j + lane < n) ? __ldg(list + j + lane) : 0;
+                    if constexpr (kDirect) cmine = __ldg(a.tile_coord + mine);
+                }
                 const int y = row0 + __shfl_sync(0xffffffffu, mine, j & 31) * 128;
+                int4 tc = make_int4(0, 0, 0, 0);
+                if constexpr (kDirect) {
+                    tc.x = __shfl_sync(0xffffffffu, cmine.x, j & 31);
+                    tc.y = __shfl_sync(0xffffffffu, cmine.y, j & 31);
+                    tc.z = __shfl_sync(0xffffffffu, cmine.z, j & 31);
+                    tc.w = __shfl_sync(0xffffffffu, cmine.w, j & 31);
+                }
                 const int st = issued % S, u = issued / S;
                 uint64_t* empty = kq ? &B.k_empty[st] : &B.v_empty[st];
                 uint64_t* full = kq ? &B.k_full[st] : &B.v_full[st];
@@ -275,8 +320,20 @@ __global__ void __launch_bounds__(384, 1)
                     if (ptx::elect_one()) {
                         ptx::mbar_arrive_expect_tx(full, bytes);
                         const int boxes = kq ? C::kBoxesQK : C::kBoxes, xstep = (kq && kFp8) ? 128 : 64;
-                        for (int x = 0; x < boxes; ++x)
-                            ptx::tma_load_2d_hint(dst + x * 16384, kq ? &tm_k : &tm_v, x * xstep, y, full, keep);
+                        for (int x = 0; x < boxes; ++x) {
+                            if constexpr (kDirect) {
+                                const AttendMaps& m = maps;
+                                if (tc.x >= 0)
+                                    ptx::tma_load_5d_hint(dst + x * 16384, kq ? &m.k[tc.x] : &m.v[tc.x], x * 64, head,
+                                                          tc.y, tc.z, tc.w, full, keep);
+                                else
+                                    ptx::tma_load_3d_hint(dst + x * 16384, kq ? &m.k[kGlobalMapSet] : &m.v[kGlobalMapSet],
+                                                          x * 64, head, tc.y, full, keep);
+                            } else {
+                                ptx::tma_load_2d_hint(dst + x * 16384, kq ? &maps.k[0] : &maps.v[0], x * xstep, y, full,
+                                                      keep);
+                            }
+                        }
                     }
                     __syncwarp();
                     ++issued;
@@ -421,6 +478,7 @@ __global__ void __launch_bounds__(384, 1)
             uint64_t lsum = ptx::f2_pack(0.f, 0.f);
             bool ok = true;
             int my_vc = 128;
+            int my_tile = 0;  // gather-free variant: the tile id, for its position mask
             float my_sk = 1.f;
             const float sq = kFp8 ? __ldg(a.scales_q + int64_t(hh) * a.n_tiles + qt) : 1.f;
             for (int k = 0; k < nw; ++k) {
@@ -428,6 +486,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int jj = 2 * (k + lane) + w;
                     const int tile = jj < n ? __ldg(list + jj) : -1;
                     my_vc = tile >= 0 ? __ldg(a.valid_count + tile) : 128;
+                    if (kDirect) my_tile = tile;
                     if (kFp8) my_sk = tile >= 0 ? __ldg(a.scales_k + int64_t(hh) * a.n_tiles + tile) : 1.f;
                 }
                 const int vc = __shfl_sync(0xffffffffu, my_vc, k & 31);
@@ -461,9 +520,18 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
                 if (vc < 128) {
+                    if constexpr (kDirect) {
+                        // box order: the tile's rows sit where its mask says (padding in place)
+                        const uint4 m = __ldg(a.tile_mask + __shfl_sync(0xffffffffu, my_tile, k & 31));
+                        const uint32_t mw[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
-                    for (int c = 0; c < 128; ++c)
-                        if (c >= vc) s[c] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 128; ++c)
+                            if (((mw[c >> 5] >> (c & 31)) & 1u) == 0) s[c] = __float_as_uint(-INFINITY);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 128; ++c)
+                            if (c >= vc) s[c] = __float_as_uint(-INFINITY);
+                    }
                 }
                 // row max: 8 independent chains of 3-input maxima
                 float mx8[8];

@@ -24,7 +24,7 @@ struct GatherArgs {
     const int32_t* heads;         // [n_heads]
     const int32_t* perm;          // [n_slots]
     const int32_t* valid_count;   // [n_tiles]
-    __nv_bfloat16* x_t;           // [n_heads, n_slots, D] (bf16 form)
+    __nv_bfloat16* x_t;           // [n_heads, n_slots, D] (bf16 form), or null: pooled features only
     uint8_t* codes;               // [n_heads, n_slots, D] 8-bit codes (kCode != 0)
     float* scales;                // [n_heads, n_tiles] (kCode != 0)
     int32_t n_tiles;
@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
     if constexpr (kCode != 0) {
         __shared__ float red8[8];
         quantize_tile<D, kCode>(v, r0, vc, red8, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
-    } else {
+    } else if (a.x_t != nullptr) {
         __nv_bfloat16* dst = a.x_t + base;
 #pragma unroll
         for (int p = 0; p < kPasses; ++p) *reinterpret_cast<uint4*>(dst + int64_t(r0 + p * kRpp) * D) = v[p];

@@ -34,7 +34,7 @@ struct DeviceState {
     bool init = false;
     int sms = 0;
     int* err = nullptr;  // device address of g_err
-    bool attend_attr[6] = {false, false, false, false, false, false};  // (head_dim 128) + 2 * Q/K format
+    bool attend_attr[8] = {};  // (head_dim 128) + 2 * Q/K format; 6 + (head_dim 128) for the gather-free variant
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -83,7 +83,9 @@ int device_copy(const veda_layout* lay, const DeviceCopy** out) {
             return r;
         };
         if ((e = up(&dc.perm, lay->perm)) != cudaSuccess || (e = up(&dc.valid_count, lay->valid_count)) != cudaSuccess ||
-            (e = up(&dc.ok_list, lay->ok_list)) != cudaSuccess || (e = up(&dc.allowed, lay->allowed)) != cudaSuccess)
+            (e = up(&dc.ok_list, lay->ok_list)) != cudaSuccess || (e = up(&dc.allowed, lay->allowed)) != cudaSuccess ||
+            (e = up(&dc.box_perm, lay->box_perm)) != cudaSuccess || (e = up(&dc.tile_coord, lay->tile_coord)) != cudaSuccess ||
+            (e = up(&dc.tile_mask, lay->tile_mask)) != cudaSuccess)
             return cuda_fail(e, "uploading the layout");
         dc.ready = true;
     }
@@ -175,6 +177,9 @@ extern "C" void veda_layout_destroy(veda_layout* layout) {
             cudaFree(dc.valid_count);
             cudaFree(dc.ok_list);
             cudaFree(dc.allowed);
+            cudaFree(dc.box_perm);
+            cudaFree(dc.tile_coord);
+            cudaFree(dc.tile_mask);
         }
     }
     if (have) cudaSetDevice(cur);
@@ -211,6 +216,45 @@ extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64
     a.h_total = h_total;
     a.err = ds->err;
     dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dim == 128)
+        gather_pool_kernel<128><<<grid, 256, 0, s>>>(a);
+    else
+        gather_pool_kernel<64><<<grid, 256, 0, s>>>(a);
+    return launch_check("gather_pool_kernel");
+}
+
+extern "C" int veda_pool(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
+                         int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, void* stream) {
+    clear_error();
+    if (!layout || !x || !heads || !feats) return fail(VEDA_ERR_INVALID, "veda_pool: NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_pool: head_dim must be 64 or 128");
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_pool: head counts must be positive");
+    if (int rc = check_strided(x_strides, x, "veda_pool x")) return rc;
+    if (!aligned16(feats)) return fail(VEDA_ERR_INVALID, "veda_pool: feats needs 16-byte alignment");
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    const veda_layout_desc& d = layout->desc;
+    if (d.n_video == 0) return VEDA_OK;
+    GatherArgs a;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.s0 = x_strides[0];
+    a.s1 = x_strides[1];
+    a.heads = heads;
+    a.perm = dc->perm;
+    a.valid_count = dc->valid_count;
+    a.x_t = nullptr;  // no tile copy: pooled features only
+    a.codes = nullptr;
+    a.scales = nullptr;
+    a.n_tiles = d.n_tiles;
+    a.feats = feats;
+    a.n_slots = d.n_slots;
+    a.n_video = d.n_video;
+    a.h_total = h_total;
+    a.err = ds->err;
+    dim3 grid(unsigned(d.n_video), unsigned(n_heads));  // video tiles only: global tiles are not pooled
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dim == 128)
         gather_pool_kernel<128><<<grid, 256, 0, s>>>(a);
@@ -361,18 +405,18 @@ extern "C" int veda_select(const veda_layout* layout, const float* scores, int32
     return launch_check("select_kernel");
 }
 
-template <int D, int kQK>
-static int launch_attend(DeviceState* ds, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const AttendArgs& a, cudaStream_t s) {
+template <int D, int kQK, bool kDirect = false>
+static int launch_attend(DeviceState* ds, const AttendMaps& maps, const AttendArgs& a, cudaStream_t s) {
     using C = AttendCfg<D, kQK>;
-    const int slot = (D == 128) + 2 * kQK;
+    const int slot = kDirect ? 6 + (D == 128) : (D == 128) + 2 * kQK;
     if (!ds->attend_attr[slot]) {
-        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        cudaError_t e = cudaFuncSetAttribute(attend_kernel<D, kQK, kDirect>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
         ds->attend_attr[slot] = true;
     }
     const int grid = std::max(1, std::min(a.n_items, ds->sms));
-    attend_kernel<D, kQK><<<grid, C::kThreads, C::kSmem, s>>>(mq, mk, mv, a);
+    attend_kernel<D, kQK, kDirect><<<grid, C::kThreads, C::kSmem, s>>>(maps, a);
     return launch_check("attend_kernel");
 }
 
@@ -397,11 +441,12 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
     if (int rc = device_state(&ds)) return rc;
     const DeviceCopy* dc;
     if (int rc = device_copy(layout, &dc)) return rc;
-    CUtensorMap mq, mk, mv;
+    AttendMaps maps;
+    std::memset(&maps, 0, sizeof maps);
     const int64_t rows = int64_t(n_heads) * d.n_slots;
-    if (int rc = make_tile_map(&mq, q, rows, dim, fp8)) return rc;
-    if (int rc = make_tile_map(&mk, k, rows, dim, fp8)) return rc;
-    if (int rc = make_tile_map(&mv, v_t, rows, dim)) return rc;
+    if (int rc = make_tile_map(&maps.q[0], q, rows, dim, fp8)) return rc;
+    if (int rc = make_tile_map(&maps.k[0], k, rows, dim, fp8)) return rc;
+    if (int rc = make_tile_map(&maps.v[0], v_t, rows, dim)) return rc;
     AttendArgs a;
     a.kept_idx = kept_idx;
     a.kept_cnt = kept_cnt;
@@ -428,10 +473,13 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
     t_hold_next_attend = false;
     a.scales_q = sq;
     a.scales_k = sk;
+    a.tile_coord = nullptr;
+    a.tile_mask = nullptr;
+    a.n_map_spans = 1;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, mq, mk, mv, a, s);
-    if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, mq, mk, mv, a, s);
-    return dim == 128 ? launch_attend<128, kQKBf16>(ds, mq, mk, mv, a, s) : launch_attend<64, kQKBf16>(ds, mq, mk, mv, a, s);
+    if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, maps, a, s);
+    if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, maps, a, s);
+    return dim == 128 ? launch_attend<128, kQKBf16>(ds, maps, a, s) : launch_attend<64, kQKBf16>(ds, maps, a, s);
 }
 
 extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
@@ -440,6 +488,119 @@ extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const voi
     clear_error();
     return attend_common(layout, q_t, k_t, nullptr, nullptr, v_t, n_heads, dim, kept_idx, kept_cnt, out, out_strides,
                          h_total, heads, stream, kQKBf16);
+}
+
+static_assert(kMapSets == kMaxDirectSpans + 1, "one map set per tiled span plus the global set");
+
+// 5D map over a packed [S, H_total, D] tensor viewed as the boxes of one tiled span: dims (D, heads, w, h,
+// t) from the span's first row, box (64, 1, sw, sh, st); positions outside the grid read as zeros.
+static int make_span_map(CUtensorMap* m, const void* x, const int64_t st[3], int32_t h_total, int dim,
+                         const DirectSpan& sp) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const char* base = static_cast<const char*>(x) + sp.start * st[0] * 2;
+    cuuint64_t gdim[5] = {cuuint64_t(dim), cuuint64_t(h_total), cuuint64_t(sp.w), cuuint64_t(sp.h), cuuint64_t(sp.t)};
+    cuuint64_t gstride[4] = {cuuint64_t(st[1]) * 2, cuuint64_t(st[0]) * 2, cuuint64_t(st[0]) * 2 * cuuint64_t(sp.w),
+                             cuuint64_t(st[0]) * 2 * cuuint64_t(sp.w) * cuuint64_t(sp.h)};
+    cuuint32_t box[5] = {64, 1, cuuint32_t(sp.sw), cuuint32_t(sp.sh), cuuint32_t(sp.st)};
+    cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<char*>(base), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled (span box) failed (" + std::to_string(int(r)) + ")");
+    return VEDA_OK;
+}
+
+// 3D map over rows [0, rows) of a packed [S, H_total, D] tensor: dims (D, heads, rows), box (64, 1, 128).
+static int make_row_map(CUtensorMap* m, const void* x, const int64_t st[3], int32_t h_total, int dim, int64_t rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[3] = {cuuint64_t(dim), cuuint64_t(h_total), cuuint64_t(std::max<int64_t>(rows, 1))};
+    cuuint64_t gstride[2] = {cuuint64_t(st[1]) * 2, cuuint64_t(st[0]) * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled (global rows) failed (" + std::to_string(int(r)) + ")");
+    return VEDA_OK;
+}
+
+extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
+                                  const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                                  int32_t h_total, int32_t dim, const int32_t* heads, int32_t n_heads,
+                                  const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                                  const int64_t out_strides[3], void* stream) {
+    clear_error();
+    const char* who = "veda_attend_direct";
+    if (!layout || !q || !k || !v || !kept_idx || !kept_cnt || !out || !heads)
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
+    if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, std::string(who) + ": head_dim must be 64 or 128");
+    if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, std::string(who) + ": head counts must be positive");
+    if (int rc = check_strided(q_strides, q, "veda_attend_direct q")) return rc;
+    if (int rc = check_strided(k_strides, k, "veda_attend_direct k")) return rc;
+    if (int rc = check_strided(v_strides, v, "veda_attend_direct v")) return rc;
+    if (int rc = check_strided(out_strides, out, "veda_attend_direct out")) return rc;
+    if (!layout->direct_ok)
+        return fail(VEDA_ERR_UNSUPPORTED, std::string(who) + ": " + layout->direct_why + "; use veda_gather + veda_attend");
+    const veda_layout_desc& d = layout->desc;
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const DeviceCopy* dc;
+    if (int rc = device_copy(layout, &dc)) return rc;
+    AttendMaps maps;
+    std::memset(&maps, 0, sizeof maps);
+    const int n_spans = int(layout->spans.size());
+    for (int i = 0; i < n_spans; ++i) {
+        const DirectSpan& sp = layout->spans[size_t(i)];
+        if (int rc = make_span_map(&maps.q[i], q, q_strides, h_total, dim, sp)) return rc;
+        if (int rc = make_span_map(&maps.k[i], k, k_strides, h_total, dim, sp)) return rc;
+        if (int rc = make_span_map(&maps.v[i], v, v_strides, h_total, dim, sp)) return rc;
+    }
+    if (d.n_global > 0) {
+        // rows past the last global row read as zeros, which masks the tail of a partial last tile
+        int64_t end = 0;
+        for (int64_t i = d.n_video; i < d.n_tiles; ++i) {
+            const int32_t c = layout->valid_count[size_t(i)];
+            if (c > 0) end = std::max<int64_t>(end, int64_t(layout->perm[size_t(i * kTile + c - 1)]) + 1);
+        }
+        if (int rc = make_row_map(&maps.q[kGlobalMapSet], q, q_strides, h_total, dim, end)) return rc;
+        if (int rc = make_row_map(&maps.k[kGlobalMapSet], k, k_strides, h_total, dim, end)) return rc;
+        if (int rc = make_row_map(&maps.v[kGlobalMapSet], v, v_strides, h_total, dim, end)) return rc;
+    }
+    AttendArgs a;
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.ok_list = dc->ok_list;
+    a.valid_count = dc->valid_count;
+    a.perm = dc->box_perm;  // box order: packed row of each box position
+    a.heads = heads;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.out_s0 = out_strides[0];
+    a.out_s1 = out_strides[1];
+    a.n_slots = d.n_slots;
+    a.max_kept = d.max_kept;
+    a.n_ok = d.n_kv_ok;
+    a.n_tiles = d.n_tiles;
+    a.n_video = d.n_video;
+    a.n_global = d.n_global;
+    a.n_heads = n_heads;
+    a.h_total = h_total;
+    a.n_items = n_heads * d.n_tiles;
+    a.scale_log2 = float((1.0 / std::sqrt(double(dim))) * 1.4426950408889634);
+    a.timeout_ns = g_timeout_ns.load();
+    a.err = ds->err;
+    a.hold_q = t_hold_next_attend ? 1 : 0;
+    t_hold_next_attend = false;
+    a.scales_q = nullptr;
+    a.scales_k = nullptr;
+    a.tile_coord = reinterpret_cast<const int4*>(dc->tile_coord);
+    a.tile_mask = reinterpret_cast<const uint4*>(dc->tile_mask);
+    a.n_map_spans = n_spans;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dim == 128 ? launch_attend<128, kQKBf16, true>(ds, maps, a, s) : launch_attend<64, kQKBf16, true>(ds, maps, a, s);
 }
 
 extern "C" int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* k_codes,

@@ -12,6 +12,14 @@ namespace veda {
 
 constexpr int kTile = VEDA_TILE;
 constexpr int kMaxDevices = 64;
+constexpr int kMaxDirectSpans = 4;  // tiled spans the gather-free attend takes (one TMA map set each)
+
+// A tiled span as the gather-free attend sees it: rows start + (t * h + y) * w + x of a (t, h, w) grid,
+// cut into (st, sh, sw) boxes.
+struct DirectSpan {
+    int64_t start;
+    int32_t t, h, w, st, sh, sw;
+};
 
 // Device copy of a layout's index data, made once per device on first use.
 struct DeviceCopy {
@@ -20,6 +28,9 @@ struct DeviceCopy {
     int32_t* valid_count = nullptr;  // [n_tiles]
     int32_t* ok_list = nullptr;      // [n_kv_ok] ascending ids of non-empty tiles
     int32_t* allowed = nullptr;      // [n_blocks * n_video]
+    int32_t* box_perm = nullptr;     // [n_slots] (gather-free attend)
+    int32_t* tile_coord = nullptr;   // [n_tiles * 4]
+    int32_t* tile_mask = nullptr;    // [n_tiles * 4] (bit patterns)
 };
 
 // Records `msg` as the calling thread's last error and returns `code`.
@@ -34,6 +45,16 @@ struct veda_layout {
     std::vector<int32_t> valid_count;  // [n_tiles]
     std::vector<int32_t> ok_list;      // [n_kv_ok]
     std::vector<int32_t> allowed;      // [n_blocks * n_video]
+    // The tiles as TMA boxes of the packed tensors, for the gather-free attend. A span tile is the 3D box
+    // of its span's grid at its origin, positions in box order (t, h, w row-major), padding left in
+    // place (positions outside the grid). A global tile is the run of 128 rows from its first row, which
+    // needs the tile's rows to be consecutive.
+    std::vector<int32_t> box_perm;    // [n_slots] packed row of each box position; -1 where the tile has no row
+    std::vector<int32_t> tile_coord;  // [n_tiles * 4] span tile {span, w0, h0, t0}; global tile {-1, row0, 0, 0}
+    std::vector<int32_t> tile_mask;   // [n_tiles * 4] bit c (word c / 32) set: box position c holds a row
+    std::vector<veda::DirectSpan> spans;  // tiled spans, in tile order
+    bool direct_ok = false;           // every global tile's rows are consecutive; spans <= kMaxDirectSpans
+    std::string direct_why;           // why not, when direct_ok is false
     mutable std::mutex mu;
     mutable veda::DeviceCopy dev[veda::kMaxDevices];
 };

@@ -78,6 +78,29 @@ void tile_span(int64_t start, const Box& grid, const Box& box, std::vector<int32
             }
 }
 
+// The same boxes in the same order as tile_span, as TMA boxes of the packed tensor: box_perm holds the
+// packed row of every box position (t, h, w row-major inside the box) and -1 outside the grid, and
+// tile_coord the box origin {span, w0, h0, t0}.
+void span_boxes(int64_t start, const Box& grid, const Box& box, int32_t span, std::vector<int32_t>& box_perm,
+                std::vector<int32_t>& tile_coord) {
+    const int64_t T = grid[0], H = grid[1], W = grid[2];
+    const int64_t nt = round_up(T, box[0]) / box[0];
+    const int64_t nh = round_up(H, box[1]) / box[1];
+    const int64_t nw = round_up(W, box[2]) / box[2];
+    for (int64_t bh = 0; bh < nh; ++bh)
+        for (int64_t bw = 0; bw < nw; ++bw)
+            for (int64_t bt = 0; bt < nt; ++bt) {
+                tile_coord.insert(tile_coord.end(),
+                                  {span, int32_t(bw * box[2]), int32_t(bh * box[1]), int32_t(bt * box[0])});
+                for (int dt = 0; dt < box[0]; ++dt)
+                    for (int dh = 0; dh < box[1]; ++dh)
+                        for (int dw = 0; dw < box[2]; ++dw) {
+                            int64_t t = bt * box[0] + dt, h = bh * box[1] + dh, w = bw * box[2] + dw;
+                            box_perm.push_back(t < T && h < H && w < W ? int32_t(start + (t * H + h) * W + w) : -1);
+                        }
+            }
+}
+
 bool budget_ok(const veda_budget& b) {
     if (b.kind == VEDA_BUDGET_RATIO) return std::isfinite(b.ratio) && b.ratio >= 0.0;
     if (b.kind == VEDA_BUDGET_TILES) return b.tiles >= 0;
@@ -177,6 +200,8 @@ extern "C" int veda_plan(const veda_span* spans, int32_t n_spans, int64_t seq_le
         std::fill(covered.begin() + s.start, covered.begin() + s.start + rows, 1);
         const size_t before = perm.size();
         tile_span(s.start, s.grid, s.box, perm);
+        span_boxes(s.start, s.grid, s.box, int32_t(i), lay->box_perm, lay->tile_coord);
+        lay->spans.push_back({s.start, s.grid[0], s.grid[1], s.grid[2], s.box[0], s.box[1], s.box[2]});
         if (i + 1 < use.size()) {
             ref_tiles += int64_t(perm.size() - before) / veda::kTile;
             ref_tokens += rows;
@@ -200,6 +225,29 @@ extern "C" int veda_plan(const veda_span* spans, int32_t n_spans, int64_t seq_le
         lay->valid_count[size_t(i)] = c;
         if (c > 0) lay->ok_list.push_back(int32_t(i));
     }
+
+    // box form of the global tiles: a run of 128 rows from the tile's first row, its own rows a prefix
+    lay->direct_ok = lay->spans.size() <= size_t(veda::kMaxDirectSpans);
+    if (!lay->direct_ok)
+        lay->direct_why = std::to_string(lay->spans.size()) + " tiled spans (the gather-free attend takes at most " +
+                          std::to_string(veda::kMaxDirectSpans) + ")";
+    for (int64_t i = n_video; i < n_tiles; ++i) {
+        const int32_t* rows = perm.data() + i * veda::kTile;
+        const int32_t c = lay->valid_count[size_t(i)];
+        const bool run = c > 0 && rows[c - 1] - rows[0] == c - 1;
+        if (!run && lay->direct_ok) {
+            lay->direct_ok = false;
+            lay->direct_why = "global tile " + std::to_string(i) + " is not a run of consecutive rows";
+        }
+        const int32_t row0 = c > 0 ? rows[0] : 0;
+        lay->tile_coord.insert(lay->tile_coord.end(), {-1, row0, 0, 0});
+        for (int j = 0; j < veda::kTile; ++j) lay->box_perm.push_back(run && j < c ? row0 + j : -1);
+    }
+    lay->tile_mask.assign(size_t(n_tiles) * 4, 0);
+    for (int64_t i = 0; i < n_tiles; ++i)
+        for (int j = 0; j < veda::kTile; ++j)
+            if (lay->box_perm[size_t(i * veda::kTile + j)] >= 0)
+                lay->tile_mask[size_t(i * 4 + j / 32)] |= int32_t(1u << (j % 32));
 
     d.seq_len = seq_len;
     d.n_slots = n_tiles * veda::kTile;
@@ -263,6 +311,18 @@ extern "C" int veda_layout_info(const veda_layout* layout, veda_layout_desc* out
     veda::clear_error();
     if (!layout || !out) return veda::fail(VEDA_ERR_INVALID, "veda_layout_info: NULL argument");
     *out = layout->desc;
+    return VEDA_OK;
+}
+
+extern "C" int veda_layout_export_direct(const veda_layout* layout, int32_t* box_perm, int32_t* tile_coord,
+                                         int32_t* tile_mask) {
+    veda::clear_error();
+    if (!layout) return veda::fail(VEDA_ERR_INVALID, "veda_layout_export_direct: NULL layout");
+    if (!layout->direct_ok)
+        return veda::fail(VEDA_ERR_UNSUPPORTED, "the gather-free attend cannot take this layout: " + layout->direct_why);
+    if (box_perm) std::copy(layout->box_perm.begin(), layout->box_perm.end(), box_perm);
+    if (tile_coord) std::copy(layout->tile_coord.begin(), layout->tile_coord.end(), tile_coord);
+    if (tile_mask) std::copy(layout->tile_mask.begin(), layout->tile_mask.end(), tile_mask);
     return VEDA_OK;
 }
 

@@ -2,8 +2,9 @@
 
 For each group of heads sharing a target tile box: plan (cached), gather Q and K to tile order with
 pooling (straight to e4m3 codes and per-tile scales in the FP8 Q/K variant), score, select, gather V,
-attend with the scatter fused. PyTorch only allocates device buffers and supplies the stream; every step
-runs in libveda's kernels.
+attend with the scatter fused. In the gather-free mode (``direct``) Q and K are only pooled and the attend
+loads every tile as a TMA box of the packed tensors, so no tile-order copy is made. PyTorch only allocates
+device buffers and supplies the stream; every step runs in libveda's kernels.
 """
 from __future__ import annotations
 
@@ -21,15 +22,21 @@ class VedaLayer:
     target       (start, (t, h, w)) the generated span (last)
     head_shapes  per head: a (t, h, w) box or None for the target's least-padding box
     budgets      (generated, reference), each a (ratio, tiles) pair with exactly one set
+    direct       gather-free attend: pool Q and K, then veda_attend_direct on the packed tensors (no
+                 tile-order copies). None (default): used when Q/K are bf16 and every group's layout has a
+                 box form (veda_layout_export_direct); True: required (raises otherwise); False: the
+                 tile-order path (veda_gather + veda_attend), which takes every layout
     """
 
-    LAUNCHES_PER_GROUP = 8  # gather q, gather k, 3 score GEMMs, select, gather v, attend
+    LAUNCHES_PER_GROUP = 7  # gather q, gather k, 2 score GEMMs, select, gather v, attend
 
     def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False,
-                 int8_qk=False):
+                 int8_qk=False, direct=None):
         self.seq_len, self.heads, self.dim = int(seq_len), int(heads), int(dim)
         if fp8_qk and int8_qk:
             raise ValueError("VedaLayer: choose one of fp8_qk and int8_qk")
+        if direct and (fp8_qk or int8_qk):
+            raise ValueError("VedaLayer: the gather-free attend reads bf16 Q/K")
         self.fp8_qk, self.int8_qk = bool(fp8_qk), bool(int8_qk)
         self.device = torch.device(device)
         lps = L.veda_least_padding_box(target[1])
@@ -37,15 +44,23 @@ class VedaLayer:
         for h, s in enumerate(head_shapes):
             groups.setdefault(tuple(lps if s is None else s), []).append(h)
         spans_ref = [(s, g, None) for s, g in ref_spans]
+        layouts = {box: L.veda_plan(spans_ref + [(target[0], target[1], box)], seq_len, budgets[0], budgets[1])
+                   for box in sorted(groups)}
+        if direct is None:
+            direct = not (fp8_qk or int8_qk) and all(L.veda_layout_has_box_form(x) for x in layouts.values())
+        elif direct:
+            for x in layouts.values():
+                if not L.veda_layout_has_box_form(x):
+                    L.veda_layout_export_direct(x)  # raises with the reason
+        self.direct = bool(direct)
         self.groups = []
         for box in sorted(groups):
-            lay = L.veda_plan(spans_ref + [(target[0], target[1], box)], seq_len, budgets[0], budgets[1])
+            lay = layouts[box]
             hs = groups[box]
             n = len(hs)
             dev = self.device
             g = dict(box=box, heads_list=hs, layout=lay,
                      heads=torch.tensor(hs, dtype=torch.int32, device=dev),
-                     v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
                      feats_q=torch.empty(n, lay.n_video, 3 * dim, dtype=torch.float32, device=dev),
                      feats_k=torch.empty(n, lay.n_video, 3 * dim, dtype=torch.float32, device=dev),
                      workspace=torch.empty(L.veda_score_workspace_bytes(lay, n, dim) // 4, dtype=torch.float32,
@@ -59,11 +74,15 @@ class VedaLayer:
                          k8=torch.empty(n, lay.n_slots, dim, dtype=code_t, device=dev),
                          sq=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev),
                          sk=torch.empty(n, lay.n_tiles, dtype=torch.float32, device=dev))
-            else:
+            elif not self.direct:
                 g.update(q_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev),
                          k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
+            if not self.direct:
+                g.update(v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
             self.groups.append(g)
-        self.launches = self.LAUNCHES_PER_GROUP * len(self.groups)
+        # launches per group: gather q, gather k, the 2 score GEMMs, select, gather v, attend (the gather-free
+        # mode: pool q, pool k, the 2 score GEMMs, select, attend)
+        self.launches = (6 if self.direct else self.LAUNCHES_PER_GROUP) * len(self.groups)
         self._side = torch.cuda.Stream(self.device)  # the V gathers
 
     def set_projections(self, proj_q, proj_k):
@@ -123,6 +142,22 @@ class VedaLayer:
         side = self._side
         for g in self.groups:
             lay = g["layout"]
+            if self.direct:
+                m = mark("pool_qk", st)
+                L.veda_pool(lay, q, g["heads"], g["feats_q"], st)
+                L.veda_pool(lay, k, g["heads"], g["feats_k"], st)
+                done(m, st)
+                m = mark("score", st)
+                L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"],
+                             st)
+                done(m, st)
+                m = mark("select", st)
+                L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], st)
+                done(m, st)
+                m = mark("attend", st)
+                L.veda_attend_direct(lay, q, k, v, g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
+                done(m, st)
+                continue
             m = mark("gather_qk", st)
             if self.fp8_qk or self.int8_qk:
                 gather = L.veda_gather_int8 if self.int8_qk else L.veda_gather_fp8

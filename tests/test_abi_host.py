@@ -133,3 +133,64 @@ def test_work_fraction_of_mixed_geometry():
         work = kept + lay.n_global * (lay.n_tiles + lay.n_video)
         frac = work / (wl.seq_len / 128) ** 2
         assert 0.105 < frac < 0.112
+
+
+def _expected_box_rows(start, grid, box):
+    """Box origins in the pages' visiting order (h-box outermost, then w-box, then t-box) and, per box, the
+    packed row of every box position (t, h, w row-major inside the box; -1 outside the grid)."""
+    T, H, W = grid
+    st, sh, sw = box
+    out = []
+    for bh in range(-(-H // sh)):
+        for bw in range(-(-W // sw)):
+            for bt in range(-(-T // st)):
+                t0, h0, w0 = bt * st, bh * sh, bw * sw
+                rows = []
+                for dt in range(st):
+                    for dh in range(sh):
+                        for dw in range(sw):
+                            t, h, w = t0 + dt, h0 + dh, w0 + dw
+                            rows.append(start + (t * H + h) * W + w if t < T and h < H and w < W else -1)
+                out.append(((t0, h0, w0), rows))
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny", "padded_tiny", "small_mixed", "small_dense", "small_d128", "mixed",
+                                  "long"])
+def test_box_form_of_the_layout(name):
+    # the gather-free attend's boxes: every tile holds the same rows as in tile order, span tiles are the
+    # grid boxes at their origins (padding in place), global tiles are runs from their first row
+    wl = V.workload(name)
+    lps = O.least_padding_shape(wl.target[1])
+    tile_refs = not O.keeps_all(wl.reference)
+    for shape, _heads in V.head_groups(wl, lambda _: lps):
+        spans = O.layer_spans(wl.ref_spans, (wl.target[0], wl.target[1], shape), tile_refs)
+        lay_o, lay_c = _plan_both(spans, wl.seq_len, wl.generated, wl.reference)
+        box_perm, coord, mask = L.veda_layout_export_direct(lay_c)
+        perm = lay_o.perm.reshape(-1, 128)
+        bp = box_perm.reshape(-1, 128)
+        bits = (mask.view(np.uint32)[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1
+        assert np.array_equal(bits.reshape(-1, 128).astype(bool), bp >= 0)
+        for i in range(lay_o.n_tiles):
+            assert sorted(bp[i][bp[i] >= 0].tolist()) == sorted(perm[i][perm[i] >= 0].tolist()), i
+        i = 0
+        for s_idx, (start, grid, box) in enumerate(spans):
+            for (t0, h0, w0), rows in _expected_box_rows(start, grid, box):
+                assert tuple(coord[i]) == (s_idx, w0, h0, t0), i
+                assert bp[i].tolist() == rows, i
+                i += 1
+        assert i == lay_o.n_video
+        for i in range(lay_o.n_video, lay_o.n_tiles):
+            c = int(lay_o.valid_count[i])
+            row0 = int(perm[i][0])
+            assert tuple(coord[i]) == (-1, row0, 0, 0)
+            assert bp[i].tolist() == [row0 + j if j < c else -1 for j in range(128)]
+
+
+def test_box_form_needs_runs_of_global_rows():
+    # two uncovered stretches that meet inside one global tile: that tile is not a run of rows
+    lay = L.veda_plan([(100, (1, 8, 16), None)], 400, (0.5, None), (1.0, None))
+    with pytest.raises(L.VedaError) as e:
+        L.veda_layout_export_direct(lay)
+    assert e.value.code == L.VEDA_ERR_UNSUPPORTED
+    assert "not a run" in str(e.value)

@@ -39,13 +39,17 @@ def built():
     _inputs.clear()
 
 
-@pytest.mark.parametrize("name", ["single", "mixed", "long", "sweep_tiles24", "sweep_r025", "sweep_r050",
-                                  "sweep_dense", "sweep_fp8", "sweep_int8"])
-def test_full_size_layer(name):
+# the layer's own path choice (gather-free wherever the layout has a box form, as bench.py runs it), and
+# the tile-order path on two of the configurations
+@pytest.mark.parametrize("name,direct", [(n, None) for n in ["single", "mixed", "long", "sweep_tiles24", "sweep_r025",
+                                                             "sweep_r050", "sweep_dense", "sweep_fp8", "sweep_int8"]]
+                         + [("single", False), ("mixed", False)])
+def test_full_size_layer(name, direct):
     wl = V.workload(name)
     x = inputs(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk)
+                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk, direct=direct)
+    assert layer.direct == (direct is None and not (wl.fp8_qk or wl.int8_qk))
     layer.set_projections(x["pq"], x["pk"])
     out = torch.full_like(x["dq"], 7.0)
     layer.forward(x["dq"], x["dk"], x["dv"], out)

@@ -400,3 +400,51 @@ def test_int8_codes_at_rounding_midpoints():
         assert np.array_equal(f32(sc).astype(np.float64), want_scales)
         got = cd.cpu().numpy().astype(np.float64).transpose(1, 0, 2)
         assert np.array_equal(got, want_codes), int((got != want_codes).sum())
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_gather_free_attend(name):
+    # veda_pool gives veda_gather's features bit for bit; veda_attend_direct, on the packed tensors and the
+    # same lists, matches the oracle within the bf16 tolerance and the tile-order attend within rounding
+    # (identical where every tile is a full box: the keys then come in the same order)
+    c = case(name)
+    wl = c.wl
+    groups = c.groups
+    q, k, v = f32(c.q), f32(c.k), f32(c.v)
+    out_t = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    out_d = out_t.clone()
+    want_out = np.zeros((wl.seq_len, wl.heads, wl.dim), np.float64)
+    all_full = True
+    for box, heads in groups:
+        res = c.run_group(box, heads, out_t)
+        lay = res["layout"]
+        fq = torch.empty_like(res["fq"])
+        L.veda_pool(lay, c.dq, res["heads"], fq)
+        L.veda_attend_direct(lay, c.dq, c.dk, c.dv, res["kept_idx"], res["kept_cnt"], out_d, res["heads"])
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        assert torch.equal(fq, res["fq"])
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        all_full &= bool((lay_o.valid_count == 128).all())
+        _, mask = oracle_kept(lay_o, f32(res["scores"]), O.column_blocks(lay_o, wl.generated, wl.reference))
+        qt, kt, vt = (O.gather(x, lay_o, heads) for x in (q, k, v))
+        o_t = O.attend_tiles(qt, kt, vt, lay_o, lambda hh, i: np.flatnonzero(mask[hh, i]))
+        O.scatter(want_out, o_t, lay_o, heads)
+    got = f32(out_d)
+    mx, mean = attention_error(got, want_out)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    diff = np.abs(got - f32(out_t)).max()
+    if all_full:
+        assert diff == 0.0, diff
+    else:
+        assert diff <= ATT_MAX_ABS, diff
+
+
+def test_gather_free_attend_rejects_layouts_without_boxes():
+    lay = L.veda_plan([(100, (1, 8, 16), None)], 400, (0.5, None), (1.0, None))
+    x = torch.zeros(400, 1, 64, dtype=torch.bfloat16, device="cuda")
+    heads = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx = torch.zeros(1, 1, lay.max_kept, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    with pytest.raises(L.VedaError) as e:
+        L.veda_attend_direct(lay, x, x, x, idx, cnt, x.clone(), heads)
+    assert e.value.code == L.VEDA_ERR_UNSUPPORTED

@@ -45,3 +45,31 @@ def test_expired_wait_is_reported_and_the_device_stays_usable():
     assert attend(out) == L.VEDA_OK
     assert torch.equal(out, want)
     assert L.veda_sync_status() == L.VEDA_OK
+
+
+def test_expired_wait_in_the_gather_free_attend():
+    # the same bounded wait on the gather-free path (its Q loads are withheld the same way)
+    c = Case("padded_tiny")
+    box, heads = c.groups[0]
+    res = c.run_group(box, heads)
+    lay = res["layout"]
+
+    def attend(out):
+        L.veda_attend_direct(lay, c.dq, c.dk, c.dv, res["kept_idx"], res["kept_cnt"], out, res["heads"])
+        return L.veda_sync_status()
+
+    want = torch.zeros_like(res["out"])
+    assert attend(want) == L.VEDA_OK
+    L.veda_set_wait_timeout_ns(20_000_000)  # 20 ms
+    try:
+        L.veda_debug_hold_next_attend()
+        t0 = time.time()
+        rc = attend(torch.zeros_like(want))
+        elapsed = time.time() - t0
+    finally:
+        L.veda_set_wait_timeout_ns(1_000_000_000)
+    assert rc == L.VEDA_ERR_TIMEOUT, L.veda_last_error()
+    assert elapsed < 5.0
+    out = torch.zeros_like(want)
+    assert attend(out) == L.VEDA_OK
+    assert torch.equal(out, want)

@@ -448,3 +448,37 @@ def test_gather_free_attend_rejects_layouts_without_boxes():
     with pytest.raises(L.VedaError) as e:
         L.veda_attend_direct(lay, x, x, x, idx, cnt, x.clone(), heads)
     assert e.value.code == L.VEDA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["small_mixed", "small_d128"])
+@pytest.mark.parametrize("direct", [False, True])
+def test_strided_views_match_contiguous(name, direct):
+    # Q/K/V and the output as views (a head slice of a wider tensor; a head-major tensor seen as [S, H, D])
+    # give bit for bit the outputs of contiguous tensors, on both attend paths; the output's other heads
+    # are left untouched
+    from learned_block_sparse_tile_b200 import VedaLayer
+    c = case(name)
+    wl = c.wl
+    S, H, D = wl.seq_len, wl.heads, wl.dim
+    layer = VedaLayer(S, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference), H, D, direct=direct)
+    layer.set_projections(c.pq, c.pk)
+    assert layer.direct == direct
+    want = torch.zeros(S, H, D, dtype=torch.bfloat16, device="cuda")
+    layer.forward(c.dq, c.dk, c.dv, want)
+
+    def wide(x):  # [S, H + 8, D] holding x in heads [0, H)
+        w = torch.full((S, H + 8, D), 3.0, dtype=x.dtype, device=x.device)
+        w[:, :H] = x
+        return w[:, :H]
+
+    def head_major(x):  # storage [H, S, D], viewed as [S, H, D]
+        return x.permute(1, 0, 2).contiguous().permute(1, 0, 2)
+
+    for view in (wide, head_major):
+        q, k, v = view(c.dq), view(c.dk), view(c.dv)
+        assert not q.is_contiguous()
+        out_wide = torch.full((S, H + 8, D), 5.0, dtype=torch.bfloat16, device="cuda")
+        layer.forward(q, k, v, out_wide[:, :H])
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        assert torch.equal(out_wide[:, :H], want), view.__name__
+        assert bool((out_wide[:, H:] == 5.0).all())

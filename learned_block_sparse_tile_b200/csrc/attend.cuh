@@ -26,6 +26,11 @@
 //                on the FMA pipe. At the end of the item the groups exchange (max, sum) per row and each
 //                writes half of the output columns: (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / sum.
 // TMEM columns: S/P of group 0 [0,128), group 1 [128,256); O of group 0 [256, 256 + D), group 1 [384, 384 + D).
+// Loads (kDirect): the tile-order variant reads head-major tile copies through 2D maps (tile t of head h
+// at rows (h N + 128 t) of [H' N, D]). The gather-free variant reads the packed [S, H, D] tensors: a span
+// tile is one 5D box (st, sh, sw, 1, 64) of its span's grid at the tile's origin, a global tile one 3D box
+// of 128 consecutive rows; a partial box keeps its padding in place, so its keys are masked by the tile's
+// 128-bit position mask instead of by count, and query rows scatter through the box-order row table.
 // Every wait is bounded: on expiry the CTA drains its in-flight copies and MMAs, frees its TMEM and
 // returns, and the host reads VEDA_ERR_TIMEOUT.
 #pragma once

@@ -420,6 +420,44 @@ static int launch_attend(DeviceState* ds, const AttendMaps& maps, const AttendAr
     return launch_check("attend_kernel");
 }
 
+// The launch arguments both attend entry points share: lists, layout tables, output, limits and the wait
+// settings (tile tables and scales are left empty; each caller sets what its variant reads).
+static AttendArgs attend_args(const veda_layout_desc& d, const DeviceCopy* dc, const DeviceState* ds,
+                              const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                              const int64_t out_strides[3], int32_t h_total, const int32_t* heads, int32_t n_heads,
+                              int32_t dim) {
+    AttendArgs a{};
+    a.kept_idx = kept_idx;
+    a.kept_cnt = kept_cnt;
+    a.ok_list = dc->ok_list;
+    a.valid_count = dc->valid_count;
+    a.perm = dc->perm;
+    a.heads = heads;
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.out_s0 = out_strides[0];
+    a.out_s1 = out_strides[1];
+    a.n_slots = d.n_slots;
+    a.max_kept = d.max_kept;
+    a.n_ok = d.n_kv_ok;
+    a.n_tiles = d.n_tiles;
+    a.n_video = d.n_video;
+    a.n_global = d.n_global;
+    a.n_heads = n_heads;
+    a.h_total = h_total;
+    a.n_items = n_heads * d.n_tiles;
+    a.scale_log2 = float((1.0 / std::sqrt(double(dim))) * 1.4426950408889634);
+    a.timeout_ns = g_timeout_ns.load();
+    a.err = ds->err;
+    a.hold_q = t_hold_next_attend ? 1 : 0;
+    t_hold_next_attend = false;
+    a.scales_q = nullptr;
+    a.scales_k = nullptr;
+    a.tile_coord = nullptr;
+    a.tile_mask = nullptr;
+    a.n_map_spans = 1;
+    return a;
+}
+
 static int attend_common(const veda_layout* layout, const void* q, const void* k, const float* sq, const float* sk,
                          const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
                          const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
@@ -447,35 +485,9 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
     if (int rc = make_tile_map(&maps.q[0], q, rows, dim, fp8)) return rc;
     if (int rc = make_tile_map(&maps.k[0], k, rows, dim, fp8)) return rc;
     if (int rc = make_tile_map(&maps.v[0], v_t, rows, dim)) return rc;
-    AttendArgs a;
-    a.kept_idx = kept_idx;
-    a.kept_cnt = kept_cnt;
-    a.ok_list = dc->ok_list;
-    a.valid_count = dc->valid_count;
-    a.perm = dc->perm;
-    a.heads = heads;
-    a.out = static_cast<__nv_bfloat16*>(out);
-    a.out_s0 = out_strides[0];
-    a.out_s1 = out_strides[1];
-    a.n_slots = d.n_slots;
-    a.max_kept = d.max_kept;
-    a.n_ok = d.n_kv_ok;
-    a.n_tiles = d.n_tiles;
-    a.n_video = d.n_video;
-    a.n_global = d.n_global;
-    a.n_heads = n_heads;
-    a.h_total = h_total;
-    a.n_items = n_heads * d.n_tiles;
-    a.scale_log2 = float((1.0 / std::sqrt(double(dim))) * 1.4426950408889634);
-    a.timeout_ns = g_timeout_ns.load();
-    a.err = ds->err;
-    a.hold_q = t_hold_next_attend ? 1 : 0;
-    t_hold_next_attend = false;
+    AttendArgs a = attend_args(d, dc, ds, kept_idx, kept_cnt, out, out_strides, h_total, heads, n_heads, dim);
     a.scales_q = sq;
     a.scales_k = sk;
-    a.tile_coord = nullptr;
-    a.tile_mask = nullptr;
-    a.n_map_spans = 1;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, maps, a, s);
     if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, maps, a, s);
@@ -570,32 +582,8 @@ extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, cons
         if (int rc = make_row_map(&maps.k[kGlobalMapSet], k, k_strides, h_total, dim, end)) return rc;
         if (int rc = make_row_map(&maps.v[kGlobalMapSet], v, v_strides, h_total, dim, end)) return rc;
     }
-    AttendArgs a;
-    a.kept_idx = kept_idx;
-    a.kept_cnt = kept_cnt;
-    a.ok_list = dc->ok_list;
-    a.valid_count = dc->valid_count;
+    AttendArgs a = attend_args(d, dc, ds, kept_idx, kept_cnt, out, out_strides, h_total, heads, n_heads, dim);
     a.perm = dc->box_perm;  // box order: packed row of each box position
-    a.heads = heads;
-    a.out = static_cast<__nv_bfloat16*>(out);
-    a.out_s0 = out_strides[0];
-    a.out_s1 = out_strides[1];
-    a.n_slots = d.n_slots;
-    a.max_kept = d.max_kept;
-    a.n_ok = d.n_kv_ok;
-    a.n_tiles = d.n_tiles;
-    a.n_video = d.n_video;
-    a.n_global = d.n_global;
-    a.n_heads = n_heads;
-    a.h_total = h_total;
-    a.n_items = n_heads * d.n_tiles;
-    a.scale_log2 = float((1.0 / std::sqrt(double(dim))) * 1.4426950408889634);
-    a.timeout_ns = g_timeout_ns.load();
-    a.err = ds->err;
-    a.hold_q = t_hold_next_attend ? 1 : 0;
-    t_hold_next_attend = false;
-    a.scales_q = nullptr;
-    a.scales_k = nullptr;
     a.tile_coord = reinterpret_cast<const int4*>(dc->tile_coord);
     a.tile_mask = reinterpret_cast<const uint4*>(dc->tile_mask);
     a.n_map_spans = n_spans;

@@ -28,7 +28,8 @@ class VedaLayer:
                  tile-order path (veda_gather + veda_attend), which takes every layout
     """
 
-    LAUNCHES_PER_GROUP = 7  # gather q, gather k, 2 score GEMMs, select, gather v, attend
+    LAUNCHES_PER_GROUP = 7  # tile-order path: gather q, gather k, 2 score GEMMs, select, gather v, attend
+    LAUNCHES_PER_GROUP_DIRECT = 6  # gather-free path: pool q, pool k, 2 score GEMMs, select, attend
 
     def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False,
                  int8_qk=False, direct=None):
@@ -80,9 +81,7 @@ class VedaLayer:
             if not self.direct:
                 g.update(v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
             self.groups.append(g)
-        # launches per group: gather q, gather k, the 2 score GEMMs, select, gather v, attend (the gather-free
-        # mode: pool q, pool k, the 2 score GEMMs, select, attend)
-        self.launches = (6 if self.direct else self.LAUNCHES_PER_GROUP) * len(self.groups)
+        self.launches = (self.LAUNCHES_PER_GROUP_DIRECT if self.direct else self.LAUNCHES_PER_GROUP) * len(self.groups)
         self._side = torch.cuda.Stream(self.device)  # the V gathers
 
     def set_projections(self, proj_q, proj_k):

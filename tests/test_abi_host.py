@@ -194,3 +194,16 @@ def test_box_form_needs_runs_of_global_rows():
         L.veda_layout_export_direct(lay)
     assert e.value.code == L.VEDA_ERR_UNSUPPORTED
     assert "not a run" in str(e.value)
+
+
+@pytest.mark.parametrize("name", ["single", "mixed", "long", "sweep_tiles24", "sweep_r025", "sweep_r050",
+                                  "sweep_dense", "single_h4"])
+def test_published_configurations_take_the_gather_free_path(name):
+    # every head group of the published configurations has a box form, so VedaLayer's default (and the
+    # bench) runs the gather-free attend on them
+    wl = V.workload(name)
+    lps = L.veda_least_padding_box(wl.target[1])
+    spans_ref = [(s, g, None) for s, g in wl.ref_spans]
+    for shape, _heads in V.head_groups(wl, lambda _: lps):
+        lay = L.veda_plan(spans_ref + [(wl.target[0], wl.target[1], shape)], wl.seq_len, wl.generated, wl.reference)
+        assert L.veda_layout_has_box_form(lay), (name, shape)

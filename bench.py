@@ -1,9 +1,13 @@
 """Benchmark of one Veda sparse-attention layer on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--workload single] [--impl veda|reference]
+               [--path auto|gathered|direct]
 
-A step is one whole layer: gather+pool Q and K, score, select, gather V, attend with the scatter fused
-(the tile plan is cached, as the pages' layout cache does). Inputs are seeded synthetic bf16 tensors of
+A step is one whole layer with the tile plan cached (as the pages' layout cache does). On the default
+path (the layer's choice: gather-free wherever every head group's layout has a box form, which holds for
+every published configuration) a step is pool Q and K, score, select, and the attend reading the tiles
+as TMA boxes of the packed tensors with the scatter fused; on the tile-order path (``--path gathered``)
+it is gather+pool Q and K, score, select, gather V, attend. Inputs are seeded synthetic bf16 tensors of
 the workload's shape, resident in HBM when the timed region starts; they total more than the 126 MB
 L2, so no flush is needed between steps. With N GPUs each rank runs its own layer (independent
 problems, weak scaling) and the time is the max over ranks.

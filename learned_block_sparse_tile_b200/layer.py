@@ -117,8 +117,9 @@ class VedaLayer:
         """q, k, v: bf16 [S, H, D] cuda (any strides the ABI accepts); out: bf16 [S, H, D], overwritten.
 
         ``events``: optional dict; CUDA event pairs recorded around each stage are appended under the stage
-        names gather_qk, score, select, gather_v and attend (the page's PhaseTimer). gather_v runs on a
-        second stream, concurrently with score and select; the others run on ``stream``."""
+        names (the page's PhaseTimer): gather_qk, score, select, gather_v and attend on the tile-order path
+        (gather_v runs on a second stream, concurrently with score and select; the others on ``stream``),
+        pool_qk, score, select and attend on the gather-free path (all on ``stream``)."""
         st = stream if stream is not None else torch.cuda.current_stream()
 
         def mark(name, on):

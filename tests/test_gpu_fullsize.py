@@ -121,3 +121,29 @@ def _sampled_error(got, want_t, lay_o, heads, q_tiles, packed=True):
             g = got[rows[real], hh, :] if packed else got[i * 128:(i + 1) * 128][real, j, :]
             errs.append(np.abs(g - want_t[i * 128:(i + 1) * 128][real, j, :]).ravel())
     return np.concatenate(errs)
+
+
+def test_full_size_paths_agree_bit_for_bit():
+    # on the 104k layer every tile is a full box, so the gather-free attend sees the keys in the same order
+    # as the tile-order one: the two paths give the same features, lists and output, bit for bit
+    wl = V.workload("single")
+    x = inputs(wl)
+    outs = []
+    for direct in (True, False):
+        layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
+                          wl.heads, wl.dim, direct=direct)
+        layer.set_projections(x["pq"], x["pk"])
+        out = torch.full_like(x["dq"], 7.0)
+        layer.forward(x["dq"], x["dk"], x["dv"], out)
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        g = layer.groups[0]
+        outs.append((out, g["feats_q"].clone(), g["feats_k"].clone(), g["kept_idx"].clone(), g["kept_cnt"].clone()))
+        del layer
+    (o1, fq1, fk1, i1, c1), (o2, fq2, fk2, i2, c2) = outs
+    assert torch.equal(fq1, fq2) and torch.equal(fk1, fk2)
+    assert torch.equal(c1, c2)
+    for h in range(c1.shape[0]):
+        for r in range(0, c1.shape[1], 37):
+            n = int(c1[h, r])
+            assert torch.equal(i1[h, r, :n], i2[h, r, :n])
+    assert torch.equal(o1, o2)

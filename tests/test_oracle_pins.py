@@ -399,6 +399,37 @@ def test_fp8_tile_scales():
     assert np.median(rel) < 0.05
 
 
+def test_fp8_attention_exact_on_grid_values():
+    # values that are e4m3 numbers times a power-of-two step, with the tile's amax at 448 steps, quantise
+    # exactly (the scale is the step, each quotient is its own e4m3 code), so the FP8 reading's attention
+    # equals plain attention; different steps per tile and head catch a scale taken from the wrong tile or
+    # head, and a scale without the 1/448 or applied to one side only fails as well
+    lay = O.build_layout([(0, (3, 10, 12), (2, 8, 8))], 360)
+    rng = np.random.default_rng(15)
+    H, D = 2, 16
+    qt = np.zeros((lay.n_tiles * 128, H, D))
+    kt = np.zeros_like(qt)
+    for arr in (qt, kt):
+        for i in range(lay.n_tiles):
+            c = lay.valid_count[i]
+            for h in range(H):
+                step = 2.0 ** -int(rng.integers(6, 12))
+                e = rng.integers(-6, 9, size=(c, D)).astype(np.float64)       # normal e4m3 exponents
+                m = rng.integers(0, 8, size=(c, D)).astype(np.float64)        # 3 mantissa bits
+                m = np.where(e == 8, np.minimum(m, 6), m)                     # at most 448 = 1.75 * 2^8
+                code = (1 + m / 8) * np.exp2(e) * np.where(rng.random((c, D)) < 0.5, -1.0, 1.0)
+                code[0, 0] = 448.0 * (1 if rng.random() < 0.5 else -1)      # the tile's amax
+                assert np.array_equal(O.veda._round_e4m3(code), code)
+                arr[i * 128:i * 128 + c, h] = code * step
+    codes, scales = O.quantize_fp8_tiles(qt, lay)
+    assert set(np.unique(np.log2(scales))) <= set(range(-11, -5))
+    vt = rng.standard_normal(qt.shape) * lay.slot_valid[:, None, None]
+    lists = lambda hh, i: np.arange(lay.n_tiles)
+    want = O.attend_tiles(qt, kt, vt, lay, lists)
+    got = O.attend_tiles_fp8(qt, kt, vt, lay, lists)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
 # ------------------------------------------------------------------------------------------ INT8 reading
 
 def test_int8_rounding_table():

@@ -508,7 +508,8 @@ def quantize_fp8_tiles(x_t, lay):
     the scale of a tile is ``amax(|x|) over its real rows / 448`` (1.0 when that is 0); the stored
     value is ``x / scale`` rounded to nearest-even e4m3 with saturation. Returns
     ``(codes as float64 [N, H', D], scales [H', n_tiles] float64)``; the dequantised value is
-    ``code * scale``. Parity unpinned beyond the e4m3 rounding rule and the scale definition.
+    ``code * scale``. Pinned by the e4m3 rounding rule, the scale definition and exact-on-grid attention;
+    that the pages' kernel used this recipe is unpinned (they do not print one).
     """
     n = lay.n_tiles
     n_heads = x_t.shape[1]

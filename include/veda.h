@@ -177,12 +177,15 @@ int veda_score(const veda_layout* layout, const float* feats_q, const float* fea
                size_t workspace_bytes, float* scores, void* stream);
 
 /* veda_score without a workspace argument, for callers that cannot allocate device memory when they
- * need the scores (inside captured graph segments, under a memory pool someone else owns, in loops where
- * an allocation is not allowed). The pages have no counterpart: this is a service of this library.
+ * need the scores: plugins whose device memory belongs to a pool the host application owns and budgets,
+ * and real-time loops where an allocation, which can block on or synchronise with the device, is not
+ * allowed. The pages have no counterpart: this is a service of this library.
  * Same inputs, outputs and arithmetic as veda_score; the projected features live in one 4 MiB array of
  * this library's device memory (1,048,576 floats, held by every GPU that loads the library until exit)
  * and heads are processed in chunks that fit it. Nothing is allocated and nothing needs to start at zero.
- * The first call on a device looks up the array's device address (make it before any stream capture).
+ * The first call on a device looks up the array's device address and keeps it for the process's life
+ * (make that call before any stream capture; after cudaDeviceReset the kept address is stale, so do not
+ * call this entry point again in that process).
  * All calls on a device share the array: calls whose kernels overlap on the GPU race and must be
  * serialised. Errors: VEDA_ERR_UNSUPPORTED when one head needs more than the array holds
  * (2 * n_video * D > 1,048,576, i.e. n_video > 4096 at D = 128); otherwise as veda_score. */

@@ -34,7 +34,10 @@ constexpr uint32_t kKeyPos = 0xFF800000u;  // key of +inf
 
 __device__ __forceinline__ uint32_t order_key(float s) {
     if (s != s) return kKeyNeg;  // NaN ranks as -inf
-    const uint32_t u = __float_as_uint(s);
+    uint32_t u = __float_as_uint(s);
+    // -0.0 and +0.0 compare equal, so they are one score and tie (the lower column first): both take the
+    // key of +0.0
+    if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -1,17 +1,22 @@
 // veda_score_noalloc: the tile-pair logits of veda_score for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc, or any allocator, at the moment they need the scores: code that
-// runs inside a captured or replayed CUDA graph segment, plugin hosts whose memory pool is owned and
-// budgeted by someone else, or real-time loops where an allocation (and the device synchronisation it
-// may cause) is not allowed. veda_score asks its caller for a workspace; this entry point instead keeps
-// that scratch (the projected query and key features) in one fixed array in this library's device
-// memory, and the caller passes only its inputs and outputs.
+// Some callers cannot call cudaMalloc, or any allocator, at the moment they need the scores: plugin hosts
+// whose device memory is owned and budgeted by the host application's own pool (a plugin may not grow it),
+// and real-time loops where an allocation is not allowed because it can block on, or synchronise with,
+// the device. veda_score asks its caller for a workspace; this entry point instead keeps that scratch (the
+// projected query and key features) in one fixed array in this library's device memory, and the caller
+// passes only its inputs and outputs.
 //
 // The scratch is a file-scope __device__ array of kScratchFloats floats (4 MiB). Every GPU that loads
 // the library holds it until the process exits. All calls on a device share it; it keeps whatever the
 // last call left there. Nothing in it must start at zero: each head chunk's projections are written in
 // full before the scores read them. Calls whose kernels overlap on the GPU (for example on two streams
 // at once) race on the array and give wrong results; serialise them.
+//
+// The first call on a device looks up the array's device address (cudaGetSymbolAddress) and keeps it for
+// the life of the process; make that first call before any stream capture. The kept address belongs to
+// the device's current context: after cudaDeviceReset (or any teardown of the primary context) it is
+// stale, so this entry point must not be called again in that process.
 #include <cuda_runtime.h>
 
 #include <algorithm>

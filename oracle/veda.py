@@ -2,7 +2,7 @@
 
 Source of every definition: the page ``veda_core.py`` (ComfyUI-FunPack node pack, "Veda sparse
 attention, the torch half"). Citations below name that page's section and function. Where the page
-is silent or ambiguous the reading adopted is stated in the docstring and listed in the design doc.
+is silent or ambiguous the reading adopted is stated in the docstring of the function it affects.
 
 Conventions
 -----------

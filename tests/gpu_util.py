@@ -88,6 +88,32 @@ def compare_lists(res, mask, lay_o):
                 raise AssertionError(f"head {h} row {r}: got {got.tolist()} want {want.tolist()}")
 
 
+def plant_signed_zero_cuts(s, lay_o, blocks, rows):
+    """Rewrites rows of fp32 scores ``s`` [H, n_video, n_video] in place so that, in every non-keeps-all
+    column block, the selection's cut falls inside a run of zeros of alternating sign: the row keeps its
+    own tile (when the block holds it), the best columns, then the lowest-column zeros. Half of the rows
+    start the run with -0.0, half with +0.0, so a selection that ranks +0.0 above -0.0 keeps other columns
+    than the (score desc, column asc) order on IEEE comparison."""
+    for blk in blocks:
+        start, stop, budget, _ = blk
+        if O.keeps_all(budget):
+            continue
+        allowed = O.allowed_per_row(lay_o, blk)
+        for r in rows:
+            cols = [c for c in range(start, stop) if lay_o.kv_ok[c] and c != r]
+            free = int(allowed[r]) - (1 if start <= r < stop else 0)
+            if free < 1 or len(cols) < free + 4:
+                continue
+            z = min(2, free)
+            top, zeros, rest = cols[:free - z], cols[free - z:free - z + 6], cols[free - z + 6:]
+            for h in range(s.shape[0]):
+                s[h, r, top] = 50.0 + np.arange(len(top), dtype=np.float32)
+                first_neg = (r + h) % 2 == 0
+                s[h, r, zeros] = [(-0.0 if (i % 2 == 0) == first_neg else 0.0) for i in range(len(zeros))]
+                s[h, r, rest] = -10.0 - np.arange(len(rest), dtype=np.float32)
+    return s
+
+
 def attention_error(got, want, valid_rows=None):
     d = np.abs(got.astype(np.float64) - want)
     if valid_rows is not None:

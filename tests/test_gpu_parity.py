@@ -9,7 +9,7 @@ from learned_block_sparse_tile_b200 import _lib as L
 from learned_block_sparse_tile_b200 import build as B
 
 from gpu_util import (ATT_MAX_ABS, ATT_MEAN_ABS, POOL_ABS, POOL_REL, SCORE_REL, Case, attention_error,
-                      compare_lists, f32, gpu_lists, oracle_kept)
+                      compare_lists, f32, gpu_lists, oracle_kept, plant_signed_zero_cuts)
 
 pytestmark = pytest.mark.gpu
 
@@ -95,10 +95,13 @@ def test_select_on_adversarial_scores():
     s[0, 2, 3] = np.inf
     s[0, 3, 4:9] = -np.inf
     s[-1, :, 0] = 3.0
+    blocks = O.column_blocks(lay_o, wl.generated, wl.reference)
+    # rows whose cut falls inside a run of -0.0 / +0.0 scores, in both column blocks
+    plant_signed_zero_cuts(s, lay_o, blocks, rows=range(4, lay.n_video, 3))
     scores = torch.from_numpy(s).cuda()
     L.veda_select(lay, scores, res["kept_idx"], res["kept_cnt"])
     assert L.veda_sync_status() == L.VEDA_OK
-    _, mask = oracle_kept(lay_o, s, O.column_blocks(lay_o, wl.generated, wl.reference))
+    _, mask = oracle_kept(lay_o, s, blocks)
     compare_lists(res, mask, lay_o)
 
 
@@ -290,7 +293,7 @@ def test_fp8_codes_at_rounding_midpoints():
 def test_select_block_widths(width):
     # one video span of exactly `width` tiles: the warp-per-row select at the edges of its register
     # tiers (16 / 32 / 64 keys per lane) and the CTA-per-row select beyond 2048 columns; scores with
-    # many ties, -inf and NaN, bit for bit against the oracle
+    # many ties, -inf, NaN and cuts inside runs of signed zeros, bit for bit against the oracle
     spans = [(0, (1, 8, 16 * width), (1, 8, 16))]
     seq_len = 128 * width
     gen, ref = (0.1, None), (1.0, None)
@@ -301,6 +304,8 @@ def test_select_block_widths(width):
     s = np.round(rng.standard_normal((1, width, width)) * 3).astype(np.float32)  # small integers: ties
     s[0, :, rng.integers(0, width, 7)] = -np.inf
     s[0, ::5, rng.integers(0, width, 3)] = np.nan
+    # rows whose cut falls inside a run of -0.0 / +0.0 scores
+    plant_signed_zero_cuts(s, lay_o, O.column_blocks(lay_o, gen, ref), rows=range(1, width, 17))
     scores = torch.from_numpy(s).cuda()
     idx = torch.full((1, width, lay.max_kept), -7, dtype=torch.int32, device="cuda")
     cnt = torch.empty(1, width, dtype=torch.int32, device="cuda")

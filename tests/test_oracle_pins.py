@@ -259,6 +259,54 @@ def test_select_ties_go_to_lower_column():
         assert set(np.flatnonzero(kept[0, r]).tolist()) == want
 
 
+def test_select_signed_zeros_are_one_score():
+    # IEEE comparison has -0.0 == +0.0: the two are the same score, so they tie and the lower column wins
+    # whichever of them carries the sign bit (torch's topk on the page compares the same way)
+    lay = O.build_layout([(0, (1, 8, 64), (1, 8, 16))], 512)  # 4 tiles
+    z, nz = 0.0, -0.0
+    s = np.array([[[5.0, nz, z, -1.0],    # own tile 0; tie of -0 (col 1) and +0 (col 2): col 1
+                   [z, 3.0, nz, -1.0],    # own tile 1; tie of +0 (col 0) and -0 (col 2): col 0
+                   [-1.0, nz, 9.0, z],    # own tile 2; tie of -0 (col 1) and +0 (col 3): col 1
+                   [z, nz, -1.0, 2.0]]],  # own tile 3; tie of +0 (col 0) and -0 (col 1): col 0
+                 dtype=np.float32)
+    assert np.signbit(s[0, 0, 1]) and not np.signbit(s[0, 0, 2])
+    kept = O.select(s, lay, O.column_blocks(lay, (None, 2), (1.0, None)))
+    want = [{0, 1}, {0, 1}, {1, 2}, {0, 3}]
+    for r in range(4):
+        assert set(np.flatnonzero(kept[0, r]).tolist()) == want[r], r
+
+
+def test_column_blocks_closed_form_with_unequal_budgets():
+    # text rows, then a reference grid (2,16,16) = 512 rows cut at (2,8,8) into 4 tiles, then a target grid
+    # (6,16,24) = 2304 rows cut at (2,8,8) into 3*2*3 = 18 tiles; reference budget 0.5, generated 0.3.
+    # Everything below is worked out by hand from the page's _per_row / _split / _bresenham.
+    assert O.least_padding_shape((2, 16, 16)) == (2, 8, 8)
+    spans = [(150, (2, 16, 16), (2, 8, 8)), (662, (6, 16, 24), (2, 8, 8))]
+    lay = O.build_layout(spans, 150 + 512 + 2304)
+    assert (lay.n_ref, lay.n_video, lay.ref_tokens, lay.target_tokens) == (4, 22, 512, 2304)
+    gen, ref = (0.3, None), (0.5, None)
+    blocks = O.column_blocks(lay, gen, ref)
+    assert blocks == [(0, 4, ref, 512), (4, 22, gen, 2304)]
+    # reference block: ideal = 512/128 = 4 tiles, ((0.5 * 4) * 4) / 4 = 2.0 -> (k_lo, k_hi, frac) = (2, 3, 0):
+    # every one of the 22 video rows keeps 2 reference tiles
+    ref_want = np.full(22, 2)
+    assert np.array_equal(O.allowed_per_row(lay, blocks[0]), ref_want)
+    # target block: ideal = 18, ((0.3 * 18) * 18) / 18 is 5.4 to within an ulp -> (5, 6, 0.4); row r gets the
+    # extra tile when floor(0.4 (r + 1)) > floor(0.4 r): rows 2, 4, 7, 9, 12, 14, 17, 19 (floor(22 * 0.4) = 8)
+    extra = {2, 4, 7, 9, 12, 14, 17, 19}
+    gen_want = np.array([5 + (r in extra) for r in range(22)])
+    assert gen_want.sum() == 5 * 22 + 8
+    assert np.array_equal(O.allowed_per_row(lay, blocks[1]), gen_want)
+    # the selection keeps exactly those counts per block (every tile holds real rows), and the own tile of
+    # each row in the block that holds it
+    rng = np.random.default_rng(4)
+    scores = rng.standard_normal((2, 22, 22)).astype(np.float32)
+    kept = O.select(scores, lay, blocks)
+    assert np.array_equal(kept[:, :, :4].sum(-1), np.broadcast_to(ref_want, (2, 22)))
+    assert np.array_equal(kept[:, :, 4:].sum(-1), np.broadcast_to(gen_want, (2, 22)))
+    assert kept[:, np.arange(22), np.arange(22)].all()
+
+
 def test_block_mask_and_index_list():
     lay = _small_layout()
     nv, n = lay.n_video, lay.n_tiles

@@ -1,9 +1,9 @@
 """The allocation-free score entry point (veda_score_noalloc) agrees with veda_score.
 
-Callers that cannot allocate device memory when they need the scores (inside captured graph segments,
-under a memory pool they do not own, in loops where allocating is not allowed) use veda_score_noalloc,
-which keeps its scratch in a fixed array of the library's own device memory instead of taking a
-workspace. This file is collected last so that a run stopping at its first failure has already run the
+Callers that cannot allocate device memory when they need the scores (plugins whose device memory
+belongs to a pool the host application owns, real-time loops where an allocation could block on the
+device) use veda_score_noalloc, which keeps its scratch in a fixed array of the library's own device
+memory instead of taking a workspace. This file is collected last so that a run stopping at its first failure has already run the
 other tests; it passes on its own in a fresh process as well as after them.
 """
 import pytest

@@ -6,7 +6,7 @@ rows, reference spans, target span and their grids), the target box of each head
 predictor projections. It holds none of the method's arithmetic and is the one module that both the
 CPU oracle's tests and the CUDA path's callers use.
 
-Recipe (fixed, documented in DESIGN.md):
+Recipe (fixed):
 
 * ``torch.Generator('cpu')`` seeds: 0 -> Q, 1 -> K, 2 -> V, 3 -> proj_q, 4 -> proj_k,
   5 -> locality bias, 6 -> text-row bias directions. Everything is drawn on the host in fp32 and

@@ -309,6 +309,15 @@ void veda_set_wait_timeout_ns(uint64_t ns);
  * VEDA_ERR_TIMEOUT. The output of that call is unspecified; the device stays usable. */
 void veda_debug_hold_next_attend(void);
 
+/* Test hook for the attend kernel's exponentials (the pages have no counterpart): evaluates, for each of
+ * n fp32 inputs x, the three forms of 2^x the library has on the device: the FMA-pipe polynomial the
+ * attend softmax uses for part of its columns (Cody-Waite reduction plus a cubic; inputs below -126 are
+ * taken as -126), the MUFU approximation (ex2.approx.ftz) it uses for the rest, and CUDA's exp2f.
+ *  x        device fp32 [n] in.
+ *  poly, mufu, exp2f_out  device fp32 [n] out (any may be NULL to skip it).
+ * Errors: VEDA_ERR_INVALID for a NULL x or negative n. */
+int veda_debug_exp2(const float* x, float* poly, float* mufu, float* exp2f_out, int64_t n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

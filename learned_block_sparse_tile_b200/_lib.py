@@ -23,7 +23,7 @@ EXPORTS = [
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
     "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
     "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8", "veda_layout_export_direct", "veda_pool",
-    "veda_attend_direct",
+    "veda_attend_direct", "veda_debug_exp2",
 ]
 
 
@@ -98,6 +98,7 @@ def lib():
         L.veda_set_wait_timeout_ns.restype = None
         L.veda_debug_hold_next_attend.argtypes = []
         L.veda_debug_hold_next_attend.restype = None
+        L.veda_debug_exp2.argtypes = [p, p, p, p, i64, vp]
         _lib = L
     return _lib
 
@@ -309,3 +310,9 @@ def veda_set_wait_timeout_ns(ns):
 def veda_debug_hold_next_attend():
     """Test hook: the calling thread's next veda_attend withholds its Q loads (its waits expire)."""
     lib().veda_debug_hold_next_attend()
+
+
+def veda_debug_exp2(x, poly=None, mufu=None, exp2f_out=None, stream=None):
+    """Test hook: the device's three forms of 2^x (attend's polynomial, the MUFU approximation, exp2f)
+    for the fp32 CUDA tensor ``x``, written to the given fp32 tensors of the same size."""
+    _check(lib().veda_debug_exp2(_ptr(x), _ptr(poly), _ptr(mufu), _ptr(exp2f_out), x.numel(), _stream(stream)))

@@ -159,6 +159,35 @@ extern "C" void veda_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns :
 
 extern "C" void veda_debug_hold_next_attend(void) { t_hold_next_attend = true; }
 
+namespace veda {
+// The three device forms of 2^x, element by element (test hook for the attend kernel's exponentials).
+__global__ void exp2_forms_kernel(const float* x, float* poly, float* mufu, float* accurate, int64_t n) {
+    const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const float v = x[i];
+    if (poly) {
+        float p0, p1;
+        ptx::f2_unpack(ptx::f2_exp2_poly(ptx::f2_pack(v, v)), p0, p1);
+        poly[i] = p0;
+    }
+    if (mufu) mufu[i] = ptx::ex2(v);
+    if (accurate) accurate[i] = exp2f(v);
+}
+}  // namespace veda
+
+extern "C" int veda_debug_exp2(const float* x, float* poly, float* mufu, float* exp2f_out, int64_t n, void* stream) {
+    clear_error();
+    if (!x || n < 0) return fail(VEDA_ERR_INVALID, "veda_debug_exp2: NULL input or negative count");
+    if (n == 0) return VEDA_OK;
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    if (blocks > 0x7fffffff) return fail(VEDA_ERR_INVALID, "veda_debug_exp2: too many elements");
+    exp2_forms_kernel<<<unsigned(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(x, poly, mufu, exp2f_out, n);
+    return launch_check("exp2_forms_kernel");
+}
+
 extern "C" int veda_device_check(void) {
     clear_error();
     DeviceState* s;

@@ -90,9 +90,18 @@ def test_full_size_layer(name, direct):
         for h in range(len(heads)):
             for r in range(lay_o.n_video):
                 assert np.array_equal(idx[h, r, :cnt[h, r]], np.flatnonzero(mask[h, r])), (h, r)
-        # attention on sampled query tiles of every head
-        q_tiles = V.sample_tiles(lay_o.n_tiles, lay_o.n_video, 3, seed=int(rng.integers(1 << 30)))
         qt, kt, vt = (O.gather(a, lay_o, heads) for a in (x["nq"], x["nk"], x["nv"]))
+        # end-to-end kept sets: the GPU's lists (from raw Q/K) against the oracle's selection on its own
+        # float64 features and scores (rounded to fp32, the page's score type); they may differ only on
+        # near-ties of the oracle's scores
+        s_o = O.logits(O.pool(qt, lay_o), O.pool(kt, lay_o), f32(x["pq"][heads]), f32(x["pk"][heads]))
+        agree, n_rows = _kept_set_agreement(idx, cnt, s_o, lay_o, wl)
+        print(f"{name} box {g['box']}: end-to-end kept sets identical on {agree} of {n_rows} rows")
+        assert agree >= 0.999 * n_rows, (agree, n_rows)
+        # attention on at least 64 sampled query tiles of every head (plus the first and last video tiles
+        # and the first and last global tiles)
+        q_tiles = V.sample_tiles(lay_o.n_tiles, lay_o.n_video, 64, seed=int(rng.integers(1 << 30)))
+        assert len(q_tiles) >= min(64, lay_o.n_tiles)
         lists = lambda hh, i: np.flatnonzero(mask[hh, i])
         attend = O.attend_tiles_fp8 if wl.fp8_qk else O.attend_tiles_int8 if wl.int8_qk else O.attend_tiles
         o_t = attend(qt, kt, vt, lay_o, lists, q_tiles=q_tiles)
@@ -104,10 +113,50 @@ def test_full_size_layer(name, direct):
             q_err = _sampled_error(o_t, o_ref, lay_o, list(range(len(heads))), q_tiles, packed=False)
             err_ref = _sampled_error(got_out, o_ref, lay_o, heads, q_tiles)
             assert err_ref.max() <= q_err.max() + ATT_MAX_ABS, (err_ref.max(), q_err.max())
-            assert err_ref.max() <= FP8_REPORT_CAP, err_ref.max()
+            bound = READING_MAX_ABS["int8" if wl.int8_qk else "fp8"]
+            assert q_err.max() <= bound and err_ref.max() <= bound + ATT_MAX_ABS, (q_err.max(), err_ref.max())
 
 
-FP8_REPORT_CAP = 1.0  # sanity cap; the e4m3 reading itself moves outputs by a few 1e-1 on this data
+# The 8-bit readings' own max-abs error against unquantised attention on this synthetic data, oracle
+# against oracle (per-tile scales; the error is the rounding of the codes, 3 mantissa bits for e4m3):
+# measured 0.25-0.30 for e4m3 and 0.07-0.08 for int8 on sampled tiles of the 104k workload. A kernel must
+# add no more than the bf16 tolerance to it.
+READING_MAX_ABS = {"fp8": 0.35, "int8": 0.12}
+
+
+def _kept_set_agreement(idx, cnt, s_o, lay_o, wl):
+    """Rows (head, video query tile) whose GPU list equals the oracle's selection on the oracle's own
+    scores ``s_o`` (float64, rounded to fp32 as the page's scores are). Every differing row must be a
+    near-tie: each column kept by one side only scores within the score tolerance of that block's cut
+    (the allowed-th best score of the row in the block, own tile first)."""
+    s32 = s_o.astype(np.float32)
+    blocks = O.column_blocks(lay_o, wl.generated, wl.reference)
+    allowed = [O.allowed_per_row(lay_o, blk) for blk in blocks]
+    mask = O.block_mask(O.select(s32, lay_o, blocks), lay_o)
+    nv = lay_o.n_video
+    agree = 0
+    for h in range(s_o.shape[0]):
+        tol = SCORE_REL * float(np.abs(s_o[h]).max())
+        for r in range(nv):
+            got = idx[h, r, :cnt[h, r]]
+            want = np.flatnonzero(mask[h, r])
+            if np.array_equal(got, want):
+                agree += 1
+                continue
+            diff = np.setxor1d(got, want)
+            for (start, stop, budget, _), allow in zip(blocks, allowed):
+                d = diff[(diff >= start) & (diff < stop)]
+                if d.size == 0:
+                    continue
+                assert not O.keeps_all(budget), (h, r, d)
+                row = s32[h, r, start:stop].astype(np.float64)
+                row[~lay_o.kv_ok[start:stop]] = -np.inf
+                if start <= r < stop:
+                    row[r - start] = np.inf
+                cut = np.sort(row)[::-1][int(allow[r]) - 1]
+                far = np.abs(s32[h, r, d].astype(np.float64) - cut) > tol
+                assert not far.any(), (h, r, d[far].tolist(), float(cut), tol)
+    return agree, s_o.shape[0] * nv
 
 
 def _sampled_error(got, want_t, lay_o, heads, q_tiles, packed=True):

@@ -1,5 +1,6 @@
-"""The N > 1 host path of bench.py on CPU: gloo ranks agree on the max-over-ranks time, and the reference
-arm prints only on rank 0 (the other ranks exit 0 without work)."""
+"""The N > 1 host path of bench.py on CPU: gloo ranks agree on the max-over-ranks time, the reference arm
+prints only on rank 0 (the other ranks exit 0 without work), ``--gpus N`` without a launcher starts N ranks
+itself, and a rank count that disagrees with ``--gpus`` is refused."""
 import os
 import subprocess
 import sys
@@ -32,7 +33,8 @@ def test_max_over_ranks_gloo():
 def test_reference_arm_prints_on_rank_zero_only():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
-                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
+                       timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
     env.update(RANK="0", LOCAL_RANK="0", WORLD_SIZE="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
@@ -41,3 +43,32 @@ def test_reference_arm_prints_on_rank_zero_only():
     import json
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
+
+
+def _env_without_ranks():
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    return env
+
+
+def test_gpus_flag_starts_its_ranks():
+    # no launcher: bench.py --gpus 2 runs itself as two ranks (torch.distributed.run on 127.0.0.1); the
+    # reference arm then prints exactly one line, from rank 0, for n_gpus = 2
+    import json
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"], env=_env_without_ranks(),
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launched_ranks():
+    env = dict(_env_without_ranks(), RANK="0", WORLD_SIZE="2", LOCAL_RANK="0", MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--gpus", "1", "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr

@@ -149,9 +149,14 @@ int veda_least_padding_box(int32_t t, int32_t h, int32_t w, int32_t box_out[3]);
  *  x_t        device bf16 [n_heads, N, D] out: x_t[h, i] = x[perm[i], heads[h]], zero on padding.
  *  feats      device fp32 [n_heads, n_video, 3D] out, or NULL to skip pooling: per video tile and head
  *             [mean | max | min] over the tile's real rows (0 for an empty tile); mean = fp32 sum / count.
+ *  row_sq     device fp32 [n_heads, S] out, or NULL: ||x||^2 of every real row, at its packed row (the
+ *             attend's logit bound takes it for Q; rows no tile holds are left as they were).
+ *  max_sq     device fp32 [n_heads] out, or NULL: the largest ||x||^2 over the head's real rows (the
+ *             attend's logit bound takes it for K); zeroed by the call before the kernel raises it.
  * D must be 64 or 128. */
 int veda_gather(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
-                int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, void* stream);
+                int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, float* row_sq,
+                float* max_sq, void* stream);
 
 /* The pooled features of veda_gather without the tile-order copy (veda_core.py, "predictor", pool): per
  * video tile and head [mean | max | min] over the tile's real rows, mean = fp32 sum / count, 0 for an
@@ -159,9 +164,12 @@ int veda_gather(const veda_layout* layout, const void* x, const int64_t x_stride
  *  x      device bf16 [S, H_total, D] with element strides x_strides[3] (S, H, D).
  *  heads  device int32 [n_heads].
  *  feats  device fp32 [n_heads, n_video, 3D] out.
+ *  row_sq, max_sq  optional norm outputs, as for veda_gather (when either is given, the call reads the
+ *         global tiles' rows too).
  * D must be 64 or 128. With veda_attend_direct this is all the scoring path needs of Q and K. */
 int veda_pool(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
-              int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, void* stream);
+              int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, float* row_sq, float* max_sq,
+              void* stream);
 
 /* Workspace bytes veda_score needs (projected features of Q and K): 2 * n_heads * n_video * D * 4. */
 size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim);
@@ -215,12 +223,19 @@ int veda_select(const veda_layout* layout, const float* scores, int32_t n_heads,
  *                 latched as VEDA_ERR_BAD_LIST).
  *  out            device bf16 [S, H_total, D] with element strides out_strides[3]: rows of this group's
  *                 heads (heads[h]) are overwritten; padding slots are dropped.
+ *  q_row_sq   device fp32 [n_heads, S] (row_sq of veda_gather/veda_pool on Q) and
+ *  k_max_sq   device fp32 [n_heads] (max_sq of veda_gather/veda_pool on K), or both NULL: a bound on every
+ *             logit of a row, sqrt(||q||^2 max ||k||^2) (Cauchy-Schwarz). Where a softmax group's first
+ *             tile leaves every row of a warp within 2^48 of that bound, its later tiles skip the row max
+ *             and the rescale of the accumulator; the result is the same softmax (the common scale of
+ *             P, O and the row sum differs, and fp32 holds it: V entries up to 2^60 in magnitude).
+ *             With NULL every tile takes its exact row max.
  * D must be 64 or 128. Runs bf16 tensor-core MMAs (tcgen05) with fp32 accumulation and an fp32 online
  * softmax; needs an sm_100 device. */
 int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
                 int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt,
                 void* out, const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
-                void* stream);
+                const float* q_row_sq, const float* k_max_sq, void* stream);
 
 /* veda_attend reading the packed tensors directly, with no tile-order copies (gather-free): every tile
  * is loaded as a TMA box of q, k and v (veda_layout_export_direct gives the boxes). Same operation as
@@ -229,13 +244,14 @@ int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, con
  *  q, k, v    device bf16 [S, H_total, D] with element strides q/k/v_strides[3] (S, H, D); bases 16-byte
  *             aligned, S and H strides multiples of 8 elements.
  *  heads      device int32 [n_heads]: the group's heads among the H_total.
- *  kept_idx/cnt, out, out_strides: as for veda_attend.
+ *  kept_idx/cnt, out, out_strides, q_row_sq, k_max_sq: as for veda_attend (the norms from veda_pool).
  * D must be 64 or 128. VEDA_ERR_UNSUPPORTED when the layout has no box form (see
  * veda_layout_export_direct); veda_gather + veda_attend take every layout. */
 int veda_attend_direct(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
                        const int64_t k_strides[3], const void* v, const int64_t v_strides[3], int32_t h_total,
                        int32_t dim, const int32_t* heads, int32_t n_heads, const int32_t* kept_idx,
-                       const int32_t* kept_cnt, void* out, const int64_t out_strides[3], void* stream);
+                       const int32_t* kept_cnt, void* out, const int64_t out_strides[3], const float* q_row_sq,
+                       const float* k_max_sq, void* stream);
 
 /* FP8 Q/K variant, step 1 (not on the pages: their kernel quantises to INT8 by a recipe they do not
  * print; this follows the FP8 e4m3 variant of the 104k budget sweep). Per (head, 128-row tile) of a

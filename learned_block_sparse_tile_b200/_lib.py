@@ -76,16 +76,17 @@ def lib():
         L.veda_layout_destroy.argtypes = [vp]
         L.veda_layout_destroy.restype = None
         L.veda_least_padding_box.argtypes = [i32, i32, i32, C.POINTER(C.c_int32)]
-        L.veda_gather.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, vp]
-        L.veda_pool.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, vp]
+        L.veda_gather.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, p, vp]
+        L.veda_pool.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
         L.veda_attend_direct.argtypes = [vp, p, C.POINTER(C.c_int64), p, C.POINTER(C.c_int64), p,
-                                         C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, C.POINTER(C.c_int64), vp]
+                                         C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, C.POINTER(C.c_int64), p,
+                                         p, vp]
         L.veda_score_workspace_bytes.argtypes = [vp, i32, i32]
         L.veda_score_workspace_bytes.restype = C.c_size_t
         L.veda_score.argtypes = [vp, p, p, i32, i32, p, p, p, C.c_size_t, p, vp]
         L.veda_score_noalloc.argtypes = [vp, p, p, i32, i32, p, p, p, vp]
         L.veda_select.argtypes = [vp, p, i32, p, p, vp]
-        L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
+        L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, p, p, vp]
         L.veda_quantize_fp8.argtypes = [vp, p, i32, i32, p, p, vp]
         L.veda_gather_fp8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
         L.veda_quantize_int8.argtypes = [vp, p, i32, i32, p, p, vp]
@@ -200,17 +201,18 @@ def veda_least_padding_box(grid):
     return tuple(out)
 
 
-def veda_gather(layout, x, heads, x_t, feats=None, stream=None):
-    """x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; x_t: bf16 [n, N, D]; feats: fp32 [n, n_video, 3D] or None."""
+def veda_gather(layout, x, heads, x_t, feats=None, stream=None, row_sq=None, max_sq=None):
+    """x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; x_t: bf16 [n, N, D]; feats: fp32 [n, n_video, 3D] or None;
+    row_sq: fp32 [n, S] or None; max_sq: fp32 [n] or None (squared row norms for the attend's logit bound)."""
     _check(lib().veda_gather(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
-                             heads.numel(), _ptr(x_t), _ptr(feats), _stream(stream)))
+                             heads.numel(), _ptr(x_t), _ptr(feats), _ptr(row_sq), _ptr(max_sq), _stream(stream)))
 
 
-def veda_pool(layout, x, heads, feats, stream=None):
+def veda_pool(layout, x, heads, feats, stream=None, row_sq=None, max_sq=None):
     """Pooled features only (no tile copy). x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; feats: fp32
-    [n, n_video, 3D]."""
+    [n, n_video, 3D]; row_sq / max_sq: optional squared row norms, as for veda_gather."""
     _check(lib().veda_pool(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads), heads.numel(),
-                           _ptr(feats), _stream(stream)))
+                           _ptr(feats), _ptr(row_sq), _ptr(max_sq), _stream(stream)))
 
 
 def veda_score_workspace_bytes(layout, n_heads, dim):
@@ -236,19 +238,21 @@ def veda_select(layout, scores, kept_idx, kept_cnt, stream=None):
                              _stream(stream)))
 
 
-def veda_attend(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, stream=None):
-    """q_t/k_t/v_t: bf16 [n, N, D]; out: bf16 [S, H, D] (strided ok); heads: int32 [n] cuda."""
+def veda_attend(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, stream=None, q_row_sq=None, k_max_sq=None):
+    """q_t/k_t/v_t: bf16 [n, N, D]; out: bf16 [S, H, D] (strided ok); heads: int32 [n] cuda; q_row_sq / k_max_sq:
+    the optional logit bound (row_sq of Q, max_sq of K from veda_gather or veda_pool)."""
     _check(lib().veda_attend(layout.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), q_t.shape[0], q_t.shape[2],
                              _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1], _ptr(heads),
-                             _stream(stream)))
+                             _ptr(q_row_sq), _ptr(k_max_sq), _stream(stream)))
 
 
-def veda_attend_direct(layout, q, k, v, kept_idx, kept_cnt, out, heads, stream=None):
+def veda_attend_direct(layout, q, k, v, kept_idx, kept_cnt, out, heads, stream=None, q_row_sq=None, k_max_sq=None):
     """veda_attend on the packed tensors (no tile-order copies). q/k/v: bf16 [S, H, D] cuda (strided ok);
-    out: bf16 [S, H, D]; heads: int32 [n] cuda."""
+    out: bf16 [S, H, D]; heads: int32 [n] cuda; q_row_sq / k_max_sq: the optional logit bound."""
     _check(lib().veda_attend_direct(layout.handle, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                     q.shape[1], q.shape[2], _ptr(heads), heads.numel(), _ptr(kept_idx),
-                                    _ptr(kept_cnt), _ptr(out), _strides(out), _stream(stream)))
+                                    _ptr(kept_cnt), _ptr(out), _strides(out), _ptr(q_row_sq), _ptr(k_max_sq),
+                                    _stream(stream)))
 
 
 def veda_gather_fp8(layout, x, heads, codes, scales, feats=None, stream=None):

@@ -81,7 +81,19 @@ struct AttendArgs {
     const int4* tile_coord;
     const uint4* tile_mask;
     int32_t n_map_spans;  // span map sets in use (the global set is used when n_global > 0)
+    // logit bound (bf16 Q/K; both null: none): ||q||^2 of every packed row and the largest ||k||^2 of each
+    // head, so that q . k <= sqrt(||q||^2 max ||k||^2) for every key the row can see (Cauchy-Schwarz)
+    const float* q_row_sq;  // [n_heads, seq_len]
+    const float* k_max_sq;  // [n_heads]
+    int64_t seq_len;
 };
+
+// With the logit bound, a softmax group takes its reference m from the exact row maxima of its first tile
+// and keeps it for the rest of the item when every row of the warp has bound - m <= kSkipLimit (log2
+// units): every later P = 2^(s - m) then stays below 2^kSkipLimit, so the row max and the rescale of O
+// are skipped without any risk of overflow (fp32 and bf16 reach 2^127; O sums at most 2^18 keys of
+// P |v|). The result is the same softmax, only the common scale of P, O and the row sum differs.
+constexpr float kSkipLimit = 48.f;
 
 // TMA maps of one launch. The tile-ordered variant uses set 0 only (2D maps over [n_heads * N, D]). The
 // gather-free variant has one set of 5D maps per tiled span over the packed tensors viewed as
@@ -479,6 +491,12 @@ __global__ void __launch_bounds__(384, 1)
                 continue;
             }
             const int nw = group_tiles(n, w);
+            // log2-domain bound on every logit of this row (padding slots need none)
+            float bound = INFINITY;
+            if (!kFp8 && a.q_row_sq != nullptr && prow >= 0)
+                bound = sqrtf(__ldg(a.q_row_sq + int64_t(hh) * a.seq_len + prow) * __ldg(a.k_max_sq + hh)) *
+                        a.scale_log2;
+            bool skip = false;  // later tiles of the item keep the first tile's reference (no row max)
             float m_ref = -INFINITY;
             uint64_t lsum = ptx::f2_pack(0.f, 0.f);
             bool ok = true;
@@ -538,25 +556,30 @@ __global__ void __launch_bounds__(384, 1)
                             if (c >= vc) s[c] = __float_as_uint(-INFINITY);
                     }
                 }
-                // row max: 8 independent chains of 3-input maxima
-                float mx8[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(__uint_as_float(s[q]), __uint_as_float(s[8 + q]));
-#pragma unroll
-                for (int c = 16; c < 128; c += 16) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        mx8[q] = ptx::max3(mx8[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
-                }
-                const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
-                                           fmaxf(mx8[6], mx8[7]));
-                const float m_new = mx * sl2;
-                const bool resc = m_new > m_ref + 8.0f;
+                bool resc = false;
                 float alpha = 1.f;
-                if (resc) {
-                    alpha = ptx::ex2(m_ref - m_new);
-                    lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
-                    m_ref = m_new;
+                if (!skip) {
+                    // row max: 8 independent chains of 3-input maxima
+                    float mx8[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(__uint_as_float(s[q]), __uint_as_float(s[8 + q]));
+#pragma unroll
+                    for (int c = 16; c < 128; c += 16) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            mx8[q] = ptx::max3(mx8[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
+                    }
+                    const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
+                                               fmaxf(mx8[6], mx8[7]));
+                    const float m_new = mx * sl2;
+                    resc = m_new > m_ref + 8.0f;
+                    if (resc) {
+                        alpha = ptx::ex2(m_ref - m_new);
+                        lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
+                        m_ref = m_new;
+                    }
+                    if (k == 0 && a.q_row_sq != nullptr)
+                        skip = __all_sync(0xffffffffu, prow < 0 || bound - m_ref <= kSkipLimit);
                 }
                 const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
                 const uint64_t negm2 = ptx::f2_pack(negm, negm);

@@ -33,6 +33,10 @@ struct GatherArgs {
     int32_t n_video;
     int32_t h_total;
     int* err;                     // latched error bits; bit 4 = head index out of range
+    // squared row norms for the attend's bound on its logits (either may be null):
+    float* row_sq;                // [n_heads, seq_len] ||x||^2 of every real row, at its packed row
+    unsigned* max_sq;             // [n_heads] largest ||x||^2 of the head's real rows (float bits; starts at 0)
+    int64_t seq_len;
 };
 
 template <int D, int kCode = 0>
@@ -59,6 +63,38 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
         const int r = r0 + p * kRpp;
         const int pr = __ldg(a.perm + int64_t(tile) * 128 + r);
         v[p] = pr >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + int64_t(pr) * a.s0)) : make_uint4(0, 0, 0, 0);
+    }
+    if (a.row_sq != nullptr || a.max_sq != nullptr) {
+        // ||x||^2 per row: each thread squares its 8 columns, the kTpr threads of a row add up
+        __shared__ unsigned cta_max;
+        if (tid == 0) cta_max = 0u;
+        __syncthreads();
+        float best = 0.f;
+#pragma unroll
+        for (int p = 0; p < kPasses; ++p) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+            }
+#pragma unroll
+            for (int off = 1; off < kTpr; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const int pr = __ldg(a.perm + int64_t(tile) * 128 + r0 + p * kRpp);
+            if (pr >= 0) {
+                if (a.row_sq != nullptr && c == 0) a.row_sq[int64_t(hh) * a.seq_len + pr] = ss;
+                best = fmaxf(best, ss);
+            }
+        }
+        if (a.max_sq != nullptr) {
+#pragma unroll
+            for (int off = kTpr; off < 32; off <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+            // non-negative floats order as their bit patterns
+            if ((tid & 31) == 0) atomicMax(&cta_max, __float_as_uint(best));
+            __syncthreads();
+            if (tid == 0) atomicMax(a.max_sq + hh, cta_max);
+        }
     }
     const int64_t base = (int64_t(hh) * a.n_slots + int64_t(tile) * 128) * D + c * 8;
     if constexpr (kCode != 0) {

@@ -215,14 +215,24 @@ extern "C" void veda_layout_destroy(veda_layout* layout) {
     delete layout;
 }
 
+// Zeroes the per-head maxima that the pool/gather kernel raises with atomicMax.
+static int clear_max_sq(float* max_sq, int32_t n_heads, cudaStream_t s) {
+    if (!max_sq) return VEDA_OK;
+    cudaError_t e = cudaMemsetAsync(max_sq, 0, size_t(n_heads) * sizeof(float), s);
+    return e == cudaSuccess ? VEDA_OK : cuda_fail(e, "cudaMemsetAsync(max_sq)");
+}
+
 extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
-                           int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, void* stream) {
+                           int32_t dim, const int32_t* heads, int32_t n_heads, void* x_t, float* feats, float* row_sq,
+                           float* max_sq, void* stream) {
     clear_error();
     if (!layout || !x || !heads || !x_t) return fail(VEDA_ERR_INVALID, "veda_gather: NULL argument");
     if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_gather: head_dim must be 64 or 128");
     if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_gather: head counts must be positive");
     if (int rc = check_strided(x_strides, x, "veda_gather x")) return rc;
     if (!aligned16(x_t) || (feats && !aligned16(feats))) return fail(VEDA_ERR_INVALID, "veda_gather: outputs need 16-byte alignment");
+    if ((row_sq && !aligned16(row_sq)) || (max_sq && !aligned16(max_sq)))
+        return fail(VEDA_ERR_INVALID, "veda_gather: norm outputs need 16-byte alignment");
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
     const DeviceCopy* dc;
@@ -244,8 +254,12 @@ extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64
     a.n_video = d.n_video;
     a.h_total = h_total;
     a.err = ds->err;
+    a.row_sq = row_sq;
+    a.max_sq = reinterpret_cast<unsigned*>(max_sq);
+    a.seq_len = d.seq_len;
     dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int rc = clear_max_sq(max_sq, n_heads, s)) return rc;
     if (dim == 128)
         gather_pool_kernel<128><<<grid, 256, 0, s>>>(a);
     else
@@ -254,19 +268,23 @@ extern "C" int veda_gather(const veda_layout* layout, const void* x, const int64
 }
 
 extern "C" int veda_pool(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
-                         int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, void* stream) {
+                         int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, float* row_sq,
+                         float* max_sq, void* stream) {
     clear_error();
     if (!layout || !x || !heads || !feats) return fail(VEDA_ERR_INVALID, "veda_pool: NULL argument");
     if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, "veda_pool: head_dim must be 64 or 128");
     if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, "veda_pool: head counts must be positive");
     if (int rc = check_strided(x_strides, x, "veda_pool x")) return rc;
     if (!aligned16(feats)) return fail(VEDA_ERR_INVALID, "veda_pool: feats needs 16-byte alignment");
+    if ((row_sq && !aligned16(row_sq)) || (max_sq && !aligned16(max_sq)))
+        return fail(VEDA_ERR_INVALID, "veda_pool: norm outputs need 16-byte alignment");
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
     const DeviceCopy* dc;
     if (int rc = device_copy(layout, &dc)) return rc;
     const veda_layout_desc& d = layout->desc;
-    if (d.n_video == 0) return VEDA_OK;
+    const bool norms = row_sq || max_sq;
+    if (d.n_video == 0 && !norms) return VEDA_OK;
     GatherArgs a;
     a.x = static_cast<const __nv_bfloat16*>(x);
     a.s0 = x_strides[0];
@@ -283,8 +301,13 @@ extern "C" int veda_pool(const veda_layout* layout, const void* x, const int64_t
     a.n_video = d.n_video;
     a.h_total = h_total;
     a.err = ds->err;
-    dim3 grid(unsigned(d.n_video), unsigned(n_heads));  // video tiles only: global tiles are not pooled
+    a.row_sq = row_sq;
+    a.max_sq = reinterpret_cast<unsigned*>(max_sq);
+    a.seq_len = d.seq_len;
+    // video tiles only (global tiles are not pooled), unless row norms are asked for: those cover every tile
+    dim3 grid(unsigned(norms ? d.n_tiles : d.n_video), unsigned(n_heads));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int rc = clear_max_sq(max_sq, n_heads, s)) return rc;
     if (dim == 128)
         gather_pool_kernel<128><<<grid, 256, 0, s>>>(a);
     else
@@ -324,6 +347,9 @@ static int gather_codes(const char* who, int code, const veda_layout* layout, co
     a.n_video = d.n_video;
     a.h_total = h_total;
     a.err = ds->err;
+    a.row_sq = nullptr;
+    a.max_sq = nullptr;
+    a.seq_len = d.seq_len;
     dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (code == kCodeI8) {
@@ -382,6 +408,31 @@ extern "C" int veda_score(const veda_layout* layout, const float* feats_q, const
     return launch_check("gemm_f32_kernel");
 }
 
+template <int kPer, bool kPrefetch>
+static int launch_rows(DeviceState* ds, const SelectArgs& a, int64_t n_rows, cudaStream_t st) {
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_rows_kernel<kPer, kPrefetch>,
+                                                                  32 * kRowsWarps, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor(select_rows_kernel)");
+    const int64_t want = (n_rows + kRowsWarps - 1) / kRowsWarps;
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(ds->sms) * std::max(per_sm, 1))));
+    select_rows_kernel<kPer, kPrefetch><<<grid, 32 * kRowsWarps, 0, st>>>(a);
+    return launch_check("select_rows_kernel");
+}
+
+static int launch_select_rows(DeviceState* ds, int per, const SelectArgs& a, int64_t n_rows, cudaStream_t st) {
+    switch (per) {
+        case 8: return launch_rows<8, true>(ds, a, n_rows, st);
+        case 16: return launch_rows<16, true>(ds, a, n_rows, st);
+        case 24: return launch_rows<24, true>(ds, a, n_rows, st);
+        case 32: return launch_rows<32, true>(ds, a, n_rows, st);
+        case 40: return launch_rows<40, false>(ds, a, n_rows, st);
+        case 48: return launch_rows<48, false>(ds, a, n_rows, st);
+        case 56: return launch_rows<56, false>(ds, a, n_rows, st);
+        default: return launch_rows<64, false>(ds, a, n_rows, st);
+    }
+}
+
 extern "C" int veda_select(const veda_layout* layout, const float* scores, int32_t n_heads, int32_t* kept_idx,
                            int32_t* kept_cnt, void* stream) {
     clear_error();
@@ -413,7 +464,15 @@ extern "C" int veda_select(const veda_layout* layout, const float* scores, int32
         a.blk_stop[b] = b < d.n_blocks ? d.blocks[b].stop : 0;
         a.blk_all[b] = b < d.n_blocks ? d.blocks[b].keeps_all : 0;
     }
+    a.n_heads = n_heads;
+    a.all_ok = 1;
+    for (int c = 0; c < d.n_video; ++c) a.all_ok &= layout->valid_count[c] > 0;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d.n_video <= 32 * 64) {
+        // persistent warps, one row at a time (rows of up to 2048 video tiles)
+        const int per = ((d.n_video + 31) / 32 + 7) / 8 * 8;  // slots per lane, a multiple of 8
+        return launch_select_rows(ds, per, a, int64_t(n_heads) * d.n_video, st);
+    }
     if (widest <= 32 * 64) {
         // one warp per row, the block's keys in registers
         const dim3 grid(unsigned((d.n_video + 7) / 8), unsigned(n_heads));
@@ -484,13 +543,17 @@ static AttendArgs attend_args(const veda_layout_desc& d, const DeviceCopy* dc, c
     a.tile_coord = nullptr;
     a.tile_mask = nullptr;
     a.n_map_spans = 1;
+    a.q_row_sq = nullptr;
+    a.k_max_sq = nullptr;
+    a.seq_len = d.seq_len;
     return a;
 }
 
 static int attend_common(const veda_layout* layout, const void* q, const void* k, const float* sq, const float* sk,
                          const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
                          const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
-                         const int32_t* heads, void* stream, int qk) {
+                         const int32_t* heads, void* stream, int qk, const float* q_row_sq = nullptr,
+                         const float* k_max_sq = nullptr) {
     const bool fp8 = qk != kQKBf16;  // 8-bit Q/K codes (e4m3 or int8)
     const char* who = qk == kQKI8 ? "veda_attend_int8" : fp8 ? "veda_attend_fp8" : "veda_attend";
     if (!layout || !q || !k || !v_t || !kept_idx || !kept_cnt || !out || !heads || (fp8 && (!sq || !sk)))
@@ -517,6 +580,10 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
     AttendArgs a = attend_args(d, dc, ds, kept_idx, kept_cnt, out, out_strides, h_total, heads, n_heads, dim);
     a.scales_q = sq;
     a.scales_k = sk;
+    if (q_row_sq && k_max_sq) {  // the logit bound (bf16 Q/K only; the 8-bit variants keep the per-tile max)
+        a.q_row_sq = q_row_sq;
+        a.k_max_sq = k_max_sq;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, maps, a, s);
     if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, maps, a, s);
@@ -525,10 +592,11 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
 
 extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
                            int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
-                           const int64_t out_strides[3], int32_t h_total, const int32_t* heads, void* stream) {
+                           const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
+                           const float* q_row_sq, const float* k_max_sq, void* stream) {
     clear_error();
     return attend_common(layout, q_t, k_t, nullptr, nullptr, v_t, n_heads, dim, kept_idx, kept_cnt, out, out_strides,
-                         h_total, heads, stream, kQKBf16);
+                         h_total, heads, stream, kQKBf16, q_row_sq, k_max_sq);
 }
 
 static_assert(kMapSets == kMaxDirectSpans + 1, "one map set per tiled span plus the global set");
@@ -573,7 +641,8 @@ extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, cons
                                   const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
                                   int32_t h_total, int32_t dim, const int32_t* heads, int32_t n_heads,
                                   const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
-                                  const int64_t out_strides[3], void* stream) {
+                                  const int64_t out_strides[3], const float* q_row_sq, const float* k_max_sq,
+                                  void* stream) {
     clear_error();
     const char* who = "veda_attend_direct";
     if (!layout || !q || !k || !v || !kept_idx || !kept_cnt || !out || !heads)
@@ -616,6 +685,10 @@ extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, cons
     a.tile_coord = reinterpret_cast<const int4*>(dc->tile_coord);
     a.tile_mask = reinterpret_cast<const uint4*>(dc->tile_mask);
     a.n_map_spans = n_spans;
+    if (q_row_sq && k_max_sq) {
+        a.q_row_sq = q_row_sq;
+        a.k_max_sq = k_max_sq;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return dim == 128 ? launch_attend<128, kQKBf16, true>(ds, maps, a, s) : launch_attend<64, kQKBf16, true>(ds, maps, a, s);
 }

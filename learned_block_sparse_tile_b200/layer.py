@@ -26,13 +26,16 @@ class VedaLayer:
                  tile-order copies). None (default): used when Q/K are bf16 and every group's layout has a
                  box form (veda_layout_export_direct); True: required (raises otherwise); False: the
                  tile-order path (veda_gather + veda_attend), which takes every layout
+    logit_bound  bf16 paths: the pool/gather of Q also writes ||q||^2 per row and that of K the largest
+                 ||k||^2 per head, and the attend takes them as its logit bound (later tiles of an item may
+                 then skip the row max; same softmax). Default True; the 8-bit paths ignore it
     """
 
     LAUNCHES_PER_GROUP = 7  # tile-order path: gather q, gather k, 2 score GEMMs, select, gather v, attend
     LAUNCHES_PER_GROUP_DIRECT = 6  # gather-free path: pool q, pool k, 2 score GEMMs, select, attend
 
     def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False,
-                 int8_qk=False, direct=None):
+                 int8_qk=False, direct=None, logit_bound=True):
         self.seq_len, self.heads, self.dim = int(seq_len), int(heads), int(dim)
         if fp8_qk and int8_qk:
             raise ValueError("VedaLayer: choose one of fp8_qk and int8_qk")
@@ -54,6 +57,7 @@ class VedaLayer:
                 if not L.veda_layout_has_box_form(x):
                     L.veda_layout_export_direct(x)  # raises with the reason
         self.direct = bool(direct)
+        self.logit_bound = bool(logit_bound) and not (self.fp8_qk or self.int8_qk)
         self.groups = []
         for box in sorted(groups):
             lay = layouts[box]
@@ -80,6 +84,11 @@ class VedaLayer:
                          k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
             if not self.direct:
                 g.update(v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
+            if self.logit_bound:
+                g.update(q_row_sq=torch.empty(n, self.seq_len, dtype=torch.float32, device=dev),
+                         k_max_sq=torch.empty(n, dtype=torch.float32, device=dev))
+            else:
+                g.update(q_row_sq=None, k_max_sq=None)
             self.groups.append(g)
         self.launches = (self.LAUNCHES_PER_GROUP_DIRECT if self.direct else self.LAUNCHES_PER_GROUP) * len(self.groups)
         self._side = torch.cuda.Stream(self.device)  # the V gathers
@@ -144,8 +153,8 @@ class VedaLayer:
             lay = g["layout"]
             if self.direct:
                 m = mark("pool_qk", st)
-                L.veda_pool(lay, q, g["heads"], g["feats_q"], st)
-                L.veda_pool(lay, k, g["heads"], g["feats_k"], st)
+                L.veda_pool(lay, q, g["heads"], g["feats_q"], st, row_sq=g["q_row_sq"])
+                L.veda_pool(lay, k, g["heads"], g["feats_k"], st, max_sq=g["k_max_sq"])
                 done(m, st)
                 m = mark("score", st)
                 L.veda_score(lay, g["feats_q"], g["feats_k"], g["proj_q"], g["proj_k"], g["workspace"], g["scores"],
@@ -155,7 +164,8 @@ class VedaLayer:
                 L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], st)
                 done(m, st)
                 m = mark("attend", st)
-                L.veda_attend_direct(lay, q, k, v, g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
+                L.veda_attend_direct(lay, q, k, v, g["kept_idx"], g["kept_cnt"], out, g["heads"], st,
+                                     q_row_sq=g["q_row_sq"], k_max_sq=g["k_max_sq"])
                 done(m, st)
                 continue
             m = mark("gather_qk", st)
@@ -164,8 +174,8 @@ class VedaLayer:
                 gather(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st)
                 gather(lay, k, g["heads"], g["k8"], g["sk"], g["feats_k"], st)
             else:
-                L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st)
-                L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st)
+                L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st, row_sq=g["q_row_sq"])
+                L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st, max_sq=g["k_max_sq"])
             done(m, st)
             qk_done = torch.cuda.Event()
             qk_done.record(st)
@@ -187,6 +197,7 @@ class VedaLayer:
                 attend = L.veda_attend_int8 if self.int8_qk else L.veda_attend_fp8
                 attend(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
             else:
-                L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
+                L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st,
+                              q_row_sq=g["q_row_sq"], k_max_sq=g["k_max_sq"])
             done(m, st)
         return out

@@ -289,10 +289,33 @@ def test_fp8_codes_at_rounding_midpoints():
         assert np.array_equal(got, want_codes), int((got != want_codes).sum())
 
 
+def test_select_two_blocks_beyond_2048_video_tiles():
+    # a reference block of 1100 tiles and a target block of 1000: rows of 2100 video tiles, each block
+    # narrow enough for the warp-per-row select that keeps one block in registers; cuts inside runs of
+    # signed zeros and exact ties, bit for bit against the oracle
+    spans = [(0, (1, 8, 16 * 1100), (1, 8, 16)), (128 * 1100, (1, 8, 16 * 1000), (1, 8, 16))]
+    seq_len = 128 * 2100
+    gen, ref = (0.05, None), (0.02, None)
+    lay = L.veda_plan(spans, seq_len, gen, ref)
+    lay_o = O.build_layout(spans, seq_len)
+    assert lay.n_video == 2100 and lay.n_ref == 1100
+    rng = np.random.default_rng(2100)
+    s = np.round(rng.standard_normal((1, 2100, 2100)) * 3).astype(np.float32)
+    s[0, ::3, rng.integers(0, 2100, 5)] = np.nan
+    blocks = O.column_blocks(lay_o, gen, ref)
+    plant_signed_zero_cuts(s, lay_o, blocks, rows=range(2, 2100, 23))
+    idx = torch.full((1, 2100, lay.max_kept), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, 2100, dtype=torch.int32, device="cuda")
+    L.veda_select(lay, torch.from_numpy(s).cuda(), idx, cnt)
+    assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+    _, mask = oracle_kept(lay_o, s, blocks)
+    compare_lists(dict(kept_idx=idx, kept_cnt=cnt), mask, lay_o)
+
+
 @pytest.mark.parametrize("width", [512, 513, 1024, 2048, 2049])
 def test_select_block_widths(width):
-    # one video span of exactly `width` tiles: the warp-per-row select at the edges of its register
-    # tiers (16 / 32 / 64 keys per lane) and the CTA-per-row select beyond 2048 columns; scores with
+    # one video span of exactly `width` tiles: the persistent warp-per-row select at the edges of its
+    # register tiers (16 / 32 / 64 slots per lane) and the CTA-per-row select beyond 2048 columns; scores with
     # many ties, -inf, NaN and cuts inside runs of signed zeros, bit for bit against the oracle
     spans = [(0, (1, 8, 16 * width), (1, 8, 16))]
     seq_len = 128 * width
@@ -487,3 +510,53 @@ def test_strided_views_match_contiguous(name, direct):
         assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
         assert torch.equal(out_wide[:, :H], want), view.__name__
         assert bool((out_wide[:, H:] == 5.0).all())
+
+
+@pytest.mark.parametrize("name", SMALL)
+@pytest.mark.parametrize("q_scale", [1.0, 16.0])
+def test_logit_bound(name, q_scale):
+    # veda_pool and veda_gather write ||q||^2 per packed row and the largest ||k||^2 per head (compared with
+    # float64 norms of the same bf16 values); with them the attend may skip the row max on an item's later
+    # tiles, which is the same softmax: both attend paths stay within the tolerance of the oracle. q_scale 16
+    # (exact in bf16) widens the gap between the bound and the first tile's maxima past the limit on most
+    # warps, so those take the exact per-tile maxima instead.
+    c = case(name)
+    wl = c.wl
+    qs = c.dq * q_scale
+    q, k, v = f32(qs), f32(c.k), f32(c.v)
+    want = np.zeros((wl.seq_len, wl.heads, wl.dim), np.float64)
+    out_d = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    out_t = out_d.clone()
+    for box, heads in c.groups:
+        res = c.run_group(box, heads)
+        lay = res["layout"]
+        n = len(heads)
+        row_sq = torch.full((n, wl.seq_len), -1.0, device="cuda")
+        max_sq = torch.full((n,), -1.0, device="cuda")
+        fq, fk = torch.empty_like(res["fq"]), torch.empty_like(res["fk"])
+        L.veda_pool(lay, qs, res["heads"], fq, row_sq=row_sq)
+        L.veda_pool(lay, c.dk, res["heads"], fk, max_sq=max_sq)
+        # the tile-order path's gather writes the same norms
+        q_t, k_t = torch.empty_like(res["q_t"]), torch.empty_like(res["k_t"])
+        row_sq_g, max_sq_g = torch.full_like(row_sq, -1.0), torch.full_like(max_sq, -1.0)
+        L.veda_gather(lay, qs, res["heads"], q_t, None, row_sq=row_sq_g)
+        L.veda_gather(lay, c.dk, res["heads"], k_t, None, max_sq=max_sq_g)
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        want_q = (q[:, heads, :].astype(np.float64) ** 2).sum(-1).T  # [n, S]
+        want_k = (k[:, heads, :].astype(np.float64) ** 2).sum(-1).max(0)  # [n]
+        for got in (row_sq, row_sq_g):
+            assert np.allclose(f32(got), want_q, rtol=1e-5, atol=0)
+        for got in (max_sq, max_sq_g):
+            assert np.allclose(f32(got), want_k, rtol=1e-5, atol=0)
+        L.veda_attend_direct(lay, qs, c.dk, c.dv, res["kept_idx"], res["kept_cnt"], out_d, res["heads"],
+                             q_row_sq=row_sq, k_max_sq=max_sq)
+        L.veda_attend(lay, q_t, k_t, res["v_t"], res["kept_idx"], res["kept_cnt"], out_t, res["heads"],
+                      q_row_sq=row_sq_g, k_max_sq=max_sq_g)
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        _, mask = oracle_kept(lay_o, f32(res["scores"]), O.column_blocks(lay_o, wl.generated, wl.reference))
+        qt, kt, vt = (O.gather(x, lay_o, heads) for x in (q, k, v))
+        O.scatter(want, O.attend_tiles(qt, kt, vt, lay_o, lambda hh, i: np.flatnonzero(mask[hh, i])), lay_o, heads)
+    for out in (out_d, out_t):
+        mx, mean = attention_error(f32(out), want)
+        assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)

@@ -94,6 +94,28 @@ typedef struct {
     veda_block_desc blocks[2];
 } veda_layout_desc;
 
+/* Row ranges of a model's packed sequence and their kinds (veda_core.py, "what the packed layout holds",
+ * describe_layout: one generated video segment, reference segments of kind cond or ref_img, and others). */
+enum { VEDA_SEG_OTHER = 0, VEDA_SEG_VIDEO = 1, VEDA_SEG_COND = 2, VEDA_SEG_REF_IMG = 3 };
+typedef struct {
+    int64_t start, stop;  /* packed rows [start, stop) */
+    int32_t kind;         /* VEDA_SEG_* */
+} veda_segment;
+
+#define VEDA_MAX_PACKED_REFS 64
+
+/* What a packed sequence holds, in the terms veda_plan takes. */
+typedef struct {
+    int64_t seq_len;
+    int64_t target_start;                       /* the video segment's first row */
+    int32_t target_grid[3];                     /* (lt, lh / 2, lw / 2) */
+    int32_t n_refs;                             /* reference segments whose rows are a verified grid */
+    int64_t ref_start[VEDA_MAX_PACKED_REFS];
+    int32_t ref_grid[VEDA_MAX_PACKED_REFS][3];
+    int32_t n_skipped;                          /* cond / ref_img segments left as global rows */
+    int32_t skipped[VEDA_MAX_PACKED_REFS];      /* their indices in the segment array */
+} veda_packed_desc;
+
 /* ------------------------------------------------------------------------------------------ host */
 
 /* Builds the tile layout of one head group (veda_core.py, "tiles", build_layout and span_tiles;
@@ -140,6 +162,29 @@ void veda_layout_destroy(veda_layout* layout);
 /* The least-padding box of a grid (veda_core.py, "tiles", least_padding_shape): among the power-of-two
  * boxes that fit the grid (all 36 if none fits), fewest tiles, then most cubic, then lexicographic. */
 int veda_least_padding_box(int32_t t, int32_t h, int32_t w, int32_t box_out[3]);
+
+/* Whether packed rows [a, b) hold a row-major T x H x W grid of positions (veda_core.py, "what the packed
+ * layout holds", _grid_of): the distinct values of each position column are the axes; their sizes must
+ * multiply to b - a and the rows must list the axes' Cartesian product in row-major order (t slowest,
+ * w fastest, each axis ascending).
+ *  position_ids  host double [>= b, 3]: (t, h, w) position of every packed row, row-major.
+ *  grid_out      receives (T, H, W) when *is_grid is set to 1; *is_grid is 0 otherwise.
+ * Errors: VEDA_ERR_INVALID for NULL pointers or a < 0, b < a. */
+int veda_grid_of(const double* position_ids, int64_t a, int64_t b, int32_t grid_out[3], int32_t* is_grid);
+
+/* The spans a model's packed sequence holds (veda_core.py, "what the packed layout holds",
+ * describe_layout), ready for veda_plan: the one video segment is the target, with grid
+ * (lt, lh / 2, lw / 2) (two-by-two spatial patches of the latent grid); a cond or ref_img segment is a
+ * reference span when its rows are a verified row-major grid (veda_grid_of on the position ids) and stays
+ * global otherwise (always correct); segments of other kinds stay global.
+ *  segments      host [n_segments]; position_ids host double [seq_len, 3], or NULL (no reference can be
+ *                verified: every cond / ref_img segment stays global).
+ *  latent        (lt, lh, lw).
+ * Errors: VEDA_ERR_INVALID for NULL segments or out, a segment outside [0, seq_len), no video segment or
+ * more than one, or a video segment whose row count is not lt * (lh / 2) * (lw / 2);
+ * VEDA_ERR_UNSUPPORTED for more than VEDA_MAX_PACKED_REFS reference segments. */
+int veda_describe_packed_layout(const veda_segment* segments, int32_t n_segments, int64_t seq_len,
+                                const int32_t latent[3], const double* position_ids, veda_packed_desc* out);
 
 /* ---------------------------------------------------------------------------------------- device */
 

@@ -23,8 +23,11 @@ EXPORTS = [
     "veda_sync_status", "veda_last_error", "veda_device_check", "veda_set_wait_timeout_ns",
     "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
     "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8", "veda_layout_export_direct", "veda_pool",
-    "veda_attend_direct", "veda_debug_exp2",
+    "veda_attend_direct", "veda_debug_exp2", "veda_grid_of", "veda_describe_packed_layout",
 ]
+
+VEDA_SEG_OTHER, VEDA_SEG_VIDEO, VEDA_SEG_COND, VEDA_SEG_REF_IMG = range(4)
+VEDA_MAX_PACKED_REFS = 64
 
 
 class VedaError(RuntimeError):
@@ -38,6 +41,17 @@ class VedaError(RuntimeError):
 class Span(C.Structure):
     _fields_ = [("start", C.c_int64), ("t", C.c_int32), ("h", C.c_int32), ("w", C.c_int32),
                 ("st", C.c_int32), ("sh", C.c_int32), ("sw", C.c_int32)]
+
+
+class Segment(C.Structure):
+    _fields_ = [("start", C.c_int64), ("stop", C.c_int64), ("kind", C.c_int32)]
+
+
+class PackedDesc(C.Structure):
+    _fields_ = [("seq_len", C.c_int64), ("target_start", C.c_int64), ("target_grid", C.c_int32 * 3),
+                ("n_refs", C.c_int32), ("ref_start", C.c_int64 * VEDA_MAX_PACKED_REFS),
+                ("ref_grid", (C.c_int32 * 3) * VEDA_MAX_PACKED_REFS), ("n_skipped", C.c_int32),
+                ("skipped", C.c_int32 * VEDA_MAX_PACKED_REFS)]
 
 
 class Budget(C.Structure):
@@ -100,6 +114,9 @@ def lib():
         L.veda_debug_hold_next_attend.argtypes = []
         L.veda_debug_hold_next_attend.restype = None
         L.veda_debug_exp2.argtypes = [p, p, p, p, i64, vp]
+        L.veda_grid_of.argtypes = [p, i64, i64, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
+        L.veda_describe_packed_layout.argtypes = [C.POINTER(Segment), i32, i64, C.POINTER(C.c_int32), p,
+                                                  C.POINTER(PackedDesc)]
         _lib = L
     return _lib
 
@@ -320,3 +337,33 @@ def veda_debug_exp2(x, poly=None, mufu=None, exp2f_out=None, stream=None):
     """Test hook: the device's three forms of 2^x (attend's polynomial, the MUFU approximation, exp2f)
     for the fp32 CUDA tensor ``x``, written to the given fp32 tensors of the same size."""
     _check(lib().veda_debug_exp2(_ptr(x), _ptr(poly), _ptr(mufu), _ptr(exp2f_out), x.numel(), _stream(stream)))
+
+
+_SEG_KINDS = {"video": VEDA_SEG_VIDEO, "cond": VEDA_SEG_COND, "ref_img": VEDA_SEG_REF_IMG}
+
+
+def _positions(position_ids):
+    return None if position_ids is None else np.ascontiguousarray(np.asarray(position_ids, dtype=np.float64))
+
+
+def veda_grid_of(position_ids, a, b):
+    """(T, H, W) when packed rows a:b hold a row-major grid of the [S, 3] position ids, else None."""
+    pos = _positions(position_ids)
+    grid, ok = (C.c_int32 * 3)(), C.c_int32()
+    _check(lib().veda_grid_of(pos.ctypes.data, int(a), int(b), grid, C.byref(ok)))
+    return tuple(grid) if ok.value else None
+
+
+def veda_describe_packed_layout(segments, latent, seq_len, position_ids=None):
+    """segments: [(start, stop, kind)] with kind "video", "cond", "ref_img" or anything else; latent: (lt, lh, lw).
+    Returns (seq_len, (target start, grid), ((ref start, grid), ...), (indices of skipped segments, ...))."""
+    arr = (Segment * max(1, len(segments)))()
+    for i, (a, b, kind) in enumerate(segments):
+        arr[i] = Segment(int(a), int(b), _SEG_KINDS.get(kind, VEDA_SEG_OTHER))
+    pos = _positions(position_ids)
+    lat = (C.c_int32 * 3)(*[int(x) for x in latent])
+    d = PackedDesc()
+    _check(lib().veda_describe_packed_layout(arr, len(segments), int(seq_len), lat,
+                                             None if pos is None else pos.ctypes.data, C.byref(d)))
+    refs = tuple((int(d.ref_start[i]), tuple(d.ref_grid[i])) for i in range(d.n_refs))
+    return int(d.seq_len), (int(d.target_start), tuple(d.target_grid)), refs, tuple(d.skipped[:d.n_skipped])

@@ -335,3 +335,82 @@ extern "C" int veda_layout_export(const veda_layout* layout, int32_t* perm, int3
     if (allowed) std::copy(layout->allowed.begin(), layout->allowed.end(), allowed);
     return VEDA_OK;
 }
+
+// veda_core.py, "what the packed layout holds", _grid_of: rows [a, b) are a row-major grid of the
+// distinct values of their three position columns.
+static bool grid_of(const double* pos, int64_t a, int64_t b, int32_t grid[3]) {
+    std::vector<double> axis[3];
+    for (int c = 0; c < 3; ++c) {
+        axis[c].reserve(size_t(b - a));
+        for (int64_t r = a; r < b; ++r) axis[c].push_back(pos[r * 3 + c]);
+        std::sort(axis[c].begin(), axis[c].end());
+        axis[c].erase(std::unique(axis[c].begin(), axis[c].end()), axis[c].end());
+    }
+    const int64_t t = int64_t(axis[0].size()), h = int64_t(axis[1].size()), w = int64_t(axis[2].size());
+    if (t * h * w != b - a) return false;
+    for (int64_t i = 0; i < b - a; ++i) {
+        const double* p = pos + (a + i) * 3;
+        if (p[0] != axis[0][size_t(i / (h * w))] || p[1] != axis[1][size_t((i / w) % h)] ||
+            p[2] != axis[2][size_t(i % w)])
+            return false;
+    }
+    grid[0] = int32_t(t);
+    grid[1] = int32_t(h);
+    grid[2] = int32_t(w);
+    return true;
+}
+
+extern "C" int veda_grid_of(const double* position_ids, int64_t a, int64_t b, int32_t grid_out[3], int32_t* is_grid) {
+    veda::clear_error();
+    if (!position_ids || !grid_out || !is_grid) return veda::fail(VEDA_ERR_INVALID, "veda_grid_of: NULL argument");
+    if (a < 0 || b < a) return veda::fail(VEDA_ERR_INVALID, "veda_grid_of: rows must satisfy 0 <= a <= b");
+    *is_grid = grid_of(position_ids, a, b, grid_out) ? 1 : 0;
+    return VEDA_OK;
+}
+
+extern "C" int veda_describe_packed_layout(const veda_segment* segments, int32_t n_segments, int64_t seq_len,
+                                           const int32_t latent[3], const double* position_ids,
+                                           veda_packed_desc* out) {
+    veda::clear_error();
+    if (!segments || !latent || !out || n_segments < 0)
+        return veda::fail(VEDA_ERR_INVALID, "veda_describe_packed_layout: NULL argument");
+    int video = -1, n_video = 0;
+    for (int32_t i = 0; i < n_segments; ++i) {
+        const veda_segment& g = segments[i];
+        if (g.start < 0 || g.stop < g.start || g.stop > seq_len)
+            return veda::fail(VEDA_ERR_INVALID, "veda_describe_packed_layout: segment " + std::to_string(i) +
+                                                    " is outside the packed rows");
+        if (g.kind == VEDA_SEG_VIDEO) {
+            video = i;
+            ++n_video;
+        }
+    }
+    if (n_video != 1)
+        return veda::fail(VEDA_ERR_INVALID, "expected one target video segment, found " + std::to_string(n_video));
+    const int32_t grid[3] = {latent[0], latent[1] / 2, latent[2] / 2};
+    if (int64_t(grid[0]) * grid[1] * grid[2] != segments[video].stop - segments[video].start)
+        return veda::fail(VEDA_ERR_INVALID, "the video segment does not match the latent grid (" +
+                                                std::to_string(grid[0]) + ", " + std::to_string(grid[1]) + ", " +
+                                                std::to_string(grid[2]) + ")");
+    veda_packed_desc d{};
+    d.seq_len = seq_len;
+    d.target_start = segments[video].start;
+    for (int c = 0; c < 3; ++c) d.target_grid[c] = grid[c];
+    for (int32_t i = 0; i < n_segments; ++i) {
+        const veda_segment& g = segments[i];
+        if (g.kind != VEDA_SEG_COND && g.kind != VEDA_SEG_REF_IMG) continue;
+        if (d.n_refs + d.n_skipped >= VEDA_MAX_PACKED_REFS)
+            return veda::fail(VEDA_ERR_UNSUPPORTED, "veda_describe_packed_layout: more than " +
+                                                        std::to_string(VEDA_MAX_PACKED_REFS) + " reference segments");
+        int32_t rg[3];
+        if (position_ids && grid_of(position_ids, g.start, g.stop, rg)) {
+            d.ref_start[d.n_refs] = g.start;
+            for (int c = 0; c < 3; ++c) d.ref_grid[d.n_refs][c] = rg[c];
+            ++d.n_refs;
+        } else {
+            d.skipped[d.n_skipped++] = i;
+        }
+    }
+    *out = d;
+    return VEDA_OK;
+}

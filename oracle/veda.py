@@ -28,7 +28,8 @@ __all__ = [
     "least_padding_shape", "span_tiles", "build_layout", "gather", "scatter", "pool", "logits",
     "column_blocks", "allowed_per_row", "select", "block_mask", "tile_index_list", "attend_tiles",
     "attend_dense_mask", "dense_attention", "attention_layer", "work_stats", "quantize_fp8_tiles",
-    "attend_tiles_fp8", "quantize_int8_tiles", "attend_tiles_int8", "layer_spans",
+    "attend_tiles_fp8", "quantize_int8_tiles", "attend_tiles_int8", "layer_spans", "grid_of",
+    "describe_packed_layout",
 ]
 
 
@@ -594,6 +595,55 @@ def attend_tiles_int8(q_t, k_t, v_t, lay, kept_lists, q_tiles=None):
 # ---------------------------------------------------------------------------------------------------
 # one layer  (veda_core.py, section "one layer": attention and its stats)
 # ---------------------------------------------------------------------------------------------------
+
+# ---------------------------------------------------------------------------------------------------
+# packed layouts  (veda_core.py, section "what the packed layout holds": _grid_of, describe_layout)
+# ---------------------------------------------------------------------------------------------------
+
+def grid_of(position_ids, a, b):
+    """``(T, H, W)`` when rows ``a:b`` hold a row-major T x H x W grid of positions, else ``None``.
+
+    veda_core.py, _grid_of: the distinct values of each of the three position columns give the axes;
+    their sizes must multiply to the row count, and the rows must list the axes' Cartesian product in
+    row-major order (t slowest, w fastest), each axis ascending.
+    """
+    pos = np.asarray(position_ids)[a:b]
+    axes = [np.unique(pos[:, i]) for i in range(3)]
+    t, h, w = (x.size for x in axes)
+    if t * h * w != b - a:
+        return None
+    want = np.stack(np.meshgrid(*axes, indexing="ij"), axis=-1).reshape(-1, 3)
+    return (t, h, w) if np.array_equal(want, pos.astype(want.dtype)) else None
+
+
+def describe_packed_layout(segments, latent, seq_len, position_ids=None):
+    """The spans a model's packed sequence holds (veda_core.py, describe_layout).
+
+    ``segments`` are ``(start, stop, kind)`` row ranges; ``latent`` is the latent grid ``(lt, lh, lw)``
+    of the generated video. There must be exactly one ``"video"`` segment, and it must hold
+    ``lt * (lh // 2) * (lw // 2)`` rows (the target grid is ``(lt, lh // 2, lw // 2)``: two-by-two spatial
+    patches). Each ``"cond"`` or ``"ref_img"`` segment becomes a reference span when its rows are a
+    verified row-major grid (``grid_of`` on the position ids), and stays global otherwise (always
+    correct); other kinds stay global. Returns ``(seq_len, (target start, target grid), ((ref start,
+    grid), ...), (skipped notes, ...))``.
+    """
+    video = [(a, b) for a, b, kind in segments if kind == "video"]
+    if len(video) != 1:
+        raise VedaError(f"expected one target video segment, found {len(video)}")
+    lt, lh, lw = (int(x) for x in latent)
+    grid = (lt, lh // 2, lw // 2)
+    if grid[0] * grid[1] * grid[2] != video[0][1] - video[0][0]:
+        raise VedaError(f"the video segment does not match the latent grid {grid}")
+    refs, skipped = [], []
+    for a, b, kind in segments:
+        if kind in ("cond", "ref_img"):
+            g = None if position_ids is None else grid_of(position_ids, a, b)
+            if g:
+                refs.append((a, g))
+            else:
+                skipped.append(f"{kind}[{a}:{b}]")
+    return int(seq_len), (video[0][0], grid), tuple(refs), tuple(skipped)
+
 
 def layer_spans(ref_spans, target, tile_refs):
     """Spans of one head group: references at their least-padding box (when tiled), target last."""

@@ -215,7 +215,8 @@ def run_veda(args, rank, world, local):
     pq, pk = V.make_projections(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
                       wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk,
-                      direct={"auto": None, "gathered": False, "direct": True}[args.path])
+                      direct={"auto": None, "gathered": False, "direct": True}[args.path],
+                      logit_bound=args.logit_bound == "on")
     direct = layer.direct
     layer.set_projections(pq, pk)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
@@ -300,6 +301,7 @@ def run_veda(args, rank, world, local):
                    "head_groups": [list(g["box"]) for g in layer.groups],
                    "attend_path": ("gather-free: Q/K pooled in place, tiles loaded as TMA boxes of the packed tensors"
                                    if direct else "tile-order copies of Q/K/V (gather), then attend"),
+                   "logit_bound": layer.logit_bound,
                    "parallelism": f"replicas x{world} (one layer per rank)",
                    "l2": "no flush: per-step inputs and outputs (2.6 GB at 104k tokens) exceed the 126 MB L2"},
         "kept_tile_tflops": round(achieved_tflops, 1),
@@ -354,6 +356,9 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "gathered", "direct"],
                     help="attend on tile-order copies (gathered), on the packed tensors as TMA boxes (direct), "
                          "or the layer's choice (auto: direct where every layout has a box form)")
+    ap.add_argument("--logit-bound", default="on", choices=["on", "off"],
+                    help="attend with the Cauchy-Schwarz logit bound (later tiles of an item may skip the row max; "
+                         "the same softmax) or with the exact row max on every tile")
     ap.add_argument("--impl", default="veda", choices=["veda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)

@@ -119,9 +119,9 @@ def test_full_size_layer(name, direct):
 
 # The 8-bit readings' own max-abs error against unquantised attention on this synthetic data, oracle
 # against oracle (per-tile scales; the error is the rounding of the codes, 3 mantissa bits for e4m3):
-# measured 0.25-0.30 for e4m3 and 0.07-0.08 for int8 on sampled tiles of the 104k workload. A kernel must
-# add no more than the bf16 tolerance to it.
-READING_MAX_ABS = {"fp8": 0.35, "int8": 0.12}
+# measured 0.25 (4 heads x 24 tiles) to 0.37 (24 heads x 64+ tiles) for e4m3 and 0.07-0.08 for int8 on the
+# 104k workload. A kernel must add no more than the bf16 tolerance to it.
+READING_MAX_ABS = {"fp8": 0.45, "int8": 0.12}
 
 
 def _kept_set_agreement(idx, cnt, s_o, lay_o, wl):

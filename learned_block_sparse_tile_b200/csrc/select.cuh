@@ -307,8 +307,8 @@ __global__ void __launch_bounds__(256) select_warp_kernel(const SelectArgs a) {
 }
 
 // ---------------------------------------------------------------------------------------------------
-// select_rows_kernel: the same selection with persistent warps, one (head, video row) at a time, for rows
-// of at most 32 kPer video tiles; each warp loads its next row's scores while it selects the current one.
+// select_rows_kernel: the same selection with one warp per (head, video row), for rows of at most 32 kPer
+// video tiles.
 //
 // Column c of the row sits in lane c % 32, slot c / 32 (ballots over a slot list columns in ascending
 // order). Per column block the warp first works on a 16-bit image of the scores: every score rounded to
@@ -321,9 +321,11 @@ __global__ void __launch_bounds__(256) select_warp_kernel(const SelectArgs a) {
 //   Phase B ranks the columns whose image equals T by their exact scores (32-bit order keys, the own tile
 //   as +inf, ties to the lower column) and keeps as many as are still needed: with at most 32 such
 //   columns lane j ranks the j-th against the others; beyond that a bisection of the exact key runs over
-//   them.
-// No block barriers: a warp owns its row. The CTA shares only a bitmap of the non-empty video tiles
-// (built once) and one 32-entry list of candidate columns per warp.
+//   them, reading their scores again.
+// The outcome of each stage is a per-lane bit mask over the slots, and the loops over slots run on those
+// masks (not unrolled), which keeps the kernel's code and register footprint small. No block barriers
+// after the start: a warp owns its row. The CTA shares a bitmap of the non-empty video tiles (built once,
+// when some tile is empty) and per warp a 32-entry candidate list and a kept-candidate mask per lane.
 constexpr int kRowsWarps = 8;  // warps per CTA
 
 __device__ __forceinline__ uint32_t h2_pack(float lo, float hi) {
@@ -354,45 +356,34 @@ __device__ __forceinline__ uint32_t h2_add(uint32_t a, uint32_t b) {
 // fp16 bits of a 16-bit order key (the inverse of: non-negative h -> h | 0x8000, negative h -> ~h)
 __device__ __forceinline__ uint32_t key16_half(uint32_t k) { return (k & 0x8000u) ? (k & 0x7FFFu) : (~k & 0xFFFFu); }
 
-constexpr uint32_t kHalfNaN = 0x7E00u;
-constexpr uint32_t kHalfPosInf = 0x7C00u;
+constexpr uint32_t kHalfNaN = 0x7E00u;       // OR-ing it into an fp16 value makes a NaN
 constexpr uint32_t kKey16NegInf = 0x03FFu;  // order key of fp16 -inf
 
-// Phase B with more than 32 candidates (columns whose fp16 image equals T): bisection of their exact keys
-// for the need-th largest, ties to the lower column. The candidates are found again from the scores (the
-// same image rule as the kernel's), so the caller keeps nothing of its own live for this rare path.
-// Returns this lane's kept candidates, bit i = slot i.
-template <int kPer>
-__device__ __noinline__ uint64_t select_wide_candidates(const SelectArgs& a, const float* srow, int row, int start,
-                                                        int stop, const uint32_t* okbits, uint32_t t2, int need) {
+// The two slot bits (low half, high half) of one fp16x2 comparison result (1.0 where true).
+__device__ __forceinline__ uint64_t pair_bits(uint32_t r) {
+    return uint64_t((r & 0xFFFFu) != 0u) | (uint64_t((r >> 16) != 0u) << 1);
+}
+
+// Phase B with more than 32 candidates (slots in `cand`): bisection of their exact keys for the need-th
+// largest, ties to the lower column, reading the scores again. Returns this lane's kept candidates.
+__device__ __noinline__ uint64_t select_wide_candidates(const float* srow, int row, uint64_t cand, int n_slots,
+                                                        int need) {
     const int lane = threadIdx.x & 31;
     const unsigned lower = (1u << lane) - 1u;
-    const uint32_t th = t2 & 0xFFFFu;
-    uint32_t key[kPer];  // exact order keys of the candidates, 0 elsewhere (every real key is above 0)
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
+    auto key_of = [&](int i) -> uint32_t {
         const int c = i * 32 + lane;
-        key[i] = 0u;
-        if (c >= start && c < stop && c < a.n_video) {
-            const float x = __ldg(srow + c);
-            const bool ok = (a.all_ok || ((okbits[i] >> lane) & 1u)) && x == x && x != -INFINITY;
-            if (c == row || ok) {
-                const float v = c == row ? INFINITY : x;
-                const uint32_t hv = h2_pack(v, v) & 0xFFFFu;
-                if (h2_set_eq(hv, th) & 0xFFFFu) key[i] = c == row ? kKeyPos : order_key(x);
-            }
-        }
-    }
+        return c == row ? kKeyPos : order_key(__ldg(srow + c));
+    };
     uint32_t thr = 0;
     bool exact = false;
     for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = thr | (1u << bit);
+        const uint32_t cv = thr | (1u << bit);
         unsigned cnt = 0;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) cnt += key[i] >= cand;
+        for (int i = 0; i < n_slots; ++i)
+            if ((cand >> i) & 1u) cnt += key_of(i) >= cv;
         const int total = int(__reduce_add_sync(0xffffffffu, cnt));
         if (total >= need) {
-            thr = cand;
+            thr = cv;
             if (total == need) {
                 exact = true;
                 break;
@@ -401,34 +392,40 @@ __device__ __noinline__ uint64_t select_wide_candidates(const SelectArgs& a, con
     }
     if (exact) {
         uint32_t lo = 0xFFFFFFFFu;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i)
-            if (key[i] >= thr) lo = min(lo, key[i]);
+        for (int i = 0; i < n_slots; ++i)
+            if ((cand >> i) & 1u) {
+                const uint32_t k = key_of(i);
+                if (k >= thr) lo = min(lo, k);
+            }
         thr = __reduce_min_sync(0xffffffffu, lo);
     }
     unsigned above = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) above += key[i] > thr;
+    for (int i = 0; i < n_slots; ++i)
+        if ((cand >> i) & 1u) above += key_of(i) > thr;
     const int need2 = need - int(__reduce_add_sync(0xffffffffu, above));
     int ties = 0;  // candidates == thr taken so far, in column order
     uint64_t kept = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        const bool is_tie = key[i] == thr;
+    for (int i = 0; i < n_slots; ++i) {
+        const bool is_c = (cand >> i) & 1u;
+        const uint32_t k = is_c ? key_of(i) : 0u;
+        const bool is_tie = is_c && k == thr;
         const unsigned tie = __ballot_sync(0xffffffffu, is_tie);
-        const bool k = key[i] > thr || (is_tie && ties + __popc(tie & lower) < need2);
+        const bool take = is_c && (k > thr || (is_tie && ties + __popc(tie & lower) < need2));
         ties += __popc(tie);
-        kept |= uint64_t(k) << i;
+        kept |= uint64_t(take) << i;
     }
     return kept;
 }
 
-template <int kPer, bool kPrefetch>
+// kTwo: the layout has two column blocks (references and target), so each block works on a masked copy of
+// the row's images; with one block (every video tile) the images are used as packed.
+template <int kPer, bool kTwo>
 __global__ void __launch_bounds__(32 * kRowsWarps) select_rows_kernel(const SelectArgs a) {
     static_assert(kPer % 2 == 0 && kPer <= 64, "slots per lane");
     constexpr int kPairs = kPer / 2;
-    __shared__ uint32_t okbits[kPer];                 // bit c: video tile c holds a real row
-    __shared__ int32_t cand_col[kRowsWarps][32];      // phase B: candidate columns, ascending
+    __shared__ uint32_t okbits[kPer];             // bit c % 32 of word c / 32: video tile c holds a real row
+    __shared__ int32_t cand_col[kRowsWarps][32];  // phase B: the first 32 candidate columns, ascending
+    __shared__ uint64_t keep_mask[kRowsWarps][32];  // phase B: per lane, the slots of its kept candidates
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const unsigned lower = (1u << lane) - 1u;
     const int nv = a.n_video;
@@ -439,82 +436,54 @@ __global__ void __launch_bounds__(32 * kRowsWarps) select_rows_kernel(const Sele
             if (__ldg(a.valid_count + c) > 0) atomicOr(&okbits[c >> 5], 1u << (c & 31));
         __syncthreads();
     }
-    const int64_t n_rows = int64_t(a.n_heads) * nv;
-    const int64_t stride = int64_t(gridDim.x) * kRowsWarps;
-    int64_t rowid = int64_t(blockIdx.x) * kRowsWarps + wib;
+    const int64_t rowid = int64_t(blockIdx.x) * kRowsWarps + wib;
+    if (rowid >= int64_t(a.n_heads) * nv) return;  // whole warps only
+    const int row = int(rowid % nv);
+    const float* srow = a.scores + rowid * nv;
+    int32_t* out = a.kept_idx + rowid * a.max_kept;
 
-    float nxt[kPer];
-    auto load_row = [&](int64_t rid) {
-        const float* srow = a.scores + rid * nv;
+    // fp16 images of the row: NaN where a column can never be kept, +inf for the own tile
+    uint32_t hrow[kPairs];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int c = i * 32 + lane;
-            nxt[i] = c < nv ? __ldg(srow + c) : __int_as_float(0x7fc00000);
+    for (int j = 0; j < kPairs; ++j) {
+        float v[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = 2 * j + u, c = i * 32 + lane;
+            const float x = c < nv ? __ldg(srow + c) : 0.f;
+            const bool ok = c < nv && (a.all_ok || ((okbits[i] >> lane) & 1u)) && x == x && x != -INFINITY;
+            v[u] = c == row ? INFINITY : ok ? x : __int_as_float(0x7fc00000);
         }
-    };
-    if (kPrefetch && rowid < n_rows) load_row(rowid);
-    for (; rowid < n_rows; rowid += stride) {
-        if (!kPrefetch) load_row(rowid);
-        const int row = int(rowid % nv);
-        const float* srow = a.scores + rowid * nv;
-        int32_t* out = a.kept_idx + rowid * a.max_kept;
-        // fp16 images of the whole row: NaN where a column can never be kept, +inf for the own tile
-        uint32_t hrow[kPairs];
-#pragma unroll
-        for (int j = 0; j < kPairs; ++j) {
-            float v[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int i = 2 * j + u, c = i * 32 + lane;
-                const float x = nxt[i];
-                const bool ok = c < nv && (a.all_ok || ((okbits[i] >> lane) & 1u)) && x == x && x != -INFINITY;
-                v[u] = c == row ? INFINITY : ok ? x : __int_as_float(0x7fc00000);
+        hrow[j] = h2_pack(v[0], v[1]);
+    }
+    int pos = 0;
+    for (int b = 0; b < (kTwo ? 2 : 1); ++b) {
+        // (selects, not a.blk_*[b]: a runtime index into the kernel arguments would copy them to the stack)
+        const int start = b ? a.blk_start[1] : a.blk_start[0], stop = b ? a.blk_stop[1] : a.blk_stop[0];
+        uint64_t take = 0;  // this lane's kept slots in the block
+        if (b ? a.blk_all[1] : a.blk_all[0]) {
+            for (int i = 0; i < kPer; ++i) {
+                const int c = i * 32 + lane;
+                take |= uint64_t(c >= start && c < stop && (a.all_ok || ((okbits[i] >> lane) & 1u))) << i;
             }
-            hrow[j] = h2_pack(v[0], v[1]);
-        }
-        if (kPrefetch && rowid + stride < n_rows) load_row(rowid + stride);  // next row's scores in flight
-        int pos = 0;
-        for (int b = 0; b < a.n_blocks; ++b) {
-            // (selects, not a.blk_*[b]: a runtime index into the kernel arguments would copy them to the stack)
-            const int start = b ? a.blk_start[1] : a.blk_start[0], stop = b ? a.blk_stop[1] : a.blk_stop[0];
-            if (b ? a.blk_all[1] : a.blk_all[0]) {
-                // every non-empty tile of the block
-#pragma unroll
-                for (int i = 0; i < kPer; ++i) {
-                    const int c = i * 32 + lane;
-                    const bool take = c >= start && c < stop && (a.all_ok || ((okbits[i] >> lane) & 1u));
-                    const unsigned bal = __ballot_sync(0xffffffffu, take);
-                    if (take) out[pos + __popc(bal & lower)] = c;
-                    pos += __popc(bal);
-                }
-                continue;
-            }
+        } else {
             const int allowed = __ldg(a.allowed + int64_t(b) * nv + row);
-            // the block's images (NaN outside it) and how many of them can be kept
+            // the block's images: NaN outside [start, stop) (a single block holds every video tile)
             uint32_t h[kPairs];
             int fin = 0;
 #pragma unroll
             for (int j = 0; j < kPairs; ++j) {
                 const int c0 = 2 * j * 32 + lane, c1 = c0 + 32;
-                const bool in0 = c0 >= start && c0 < stop, in1 = c1 >= start && c1 < stop;
-                const uint32_t x = hrow[j];
-                h[j] = (in0 ? (x & 0xFFFFu) : kHalfNaN) | (in1 ? (x & 0xFFFF0000u) : (kHalfNaN << 16));
-                const uint32_t e = h2_set_eq(h[j], h[j]);  // not NaN
-                fin += ((e & 0xFFFFu) != 0u) + ((e >> 16) != 0u);
+                h[j] = kTwo ? hrow[j] | ((c0 >= start && c0 < stop) ? 0u : kHalfNaN) |
+                                  ((c1 >= start && c1 < stop) ? 0u : (kHalfNaN << 16))
+                            : hrow[j];
+                fin += __popcll(pair_bits(h2_set_eq(h[j], h[j])));  // not NaN
             }
             const int n_fin = int(__reduce_add_sync(0xffffffffu, uint32_t(fin)));
-            // mode 0: keep the images >= t2 (all keepable columns when the budget covers them, or an exact
-            // split); mode 1: images > t2, plus the phase B picks among the images == t2
-            uint32_t t2;
-            int mode = 0;
-            uint32_t keep_bits = 0;  // mode 1, at most 32 candidates: bit j = the j-th candidate is kept
-            bool wide = false;       // mode 1 with more than 32 candidates: exact-key bisection
-            uint64_t wide_keep = 0;  // wide: this lane's kept candidates, bit i = slot i
-            if (allowed <= 0) {
-                t2 = kHalfNaN | (kHalfNaN << 16);  // nothing compares >= NaN: nothing is kept
-            } else if (allowed >= n_fin) {
-                t2 = 0xFC00FC00u;  // fp16 -inf: every image that is not NaN is >= it
-            } else {
+            if (allowed >= n_fin) {
+#pragma unroll
+                for (int j = 0; j < kPairs; ++j) take |= pair_bits(h2_set_eq(h[j], h[j])) << (2 * j);
+            } else if (allowed > 0) {
                 // phase A: the largest 16-bit key whose image has at least `allowed` images >= it
                 uint32_t thr = 0;
                 bool exact = false;
@@ -522,14 +491,12 @@ __global__ void __launch_bounds__(32 * kRowsWarps) select_rows_kernel(const Sele
                     const uint32_t cand = thr | (1u << bit);
                     const uint32_t hv = key16_half(cand);
                     const uint32_t c2 = hv | (hv << 16);
-                    uint32_t acc0 = 0x64006400u, acc1 = 0x64006400u;  // 1024.0: the count sits in the low bits
+                    uint32_t acc[4] = {0x64006400u, 0x64006400u, 0x64006400u, 0x64006400u};  // 1024.0 + count
 #pragma unroll
-                    for (int j = 0; j < kPairs; j += 2) {
-                        acc0 = h2_add(acc0, h2_set_ge(h[j], c2));
-                        if (j + 1 < kPairs) acc1 = h2_add(acc1, h2_set_ge(h[j + 1], c2));
-                    }
-                    const uint32_t cnt = (acc0 & 0x3FFu) + ((acc0 >> 16) & 0x3FFu) + (acc1 & 0x3FFu) +
-                                         ((acc1 >> 16) & 0x3FFu);
+                    for (int j = 0; j < kPairs; ++j) acc[j & 3] = h2_add(acc[j & 3], h2_set_ge(h[j], c2));
+                    uint32_t cnt = 0;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) cnt += (acc[q] & 0x3FFu) + ((acc[q] >> 16) & 0x3FFu);
                     const int total = int(__reduce_add_sync(0xffffffffu, cnt));
                     if (total >= allowed) {
                         thr = cand;
@@ -543,36 +510,36 @@ __global__ void __launch_bounds__(32 * kRowsWarps) select_rows_kernel(const Sele
                 // fails, the allowed-th largest image is -inf itself
                 if (thr < kKey16NegInf) thr = kKey16NegInf;
                 const uint32_t hv = key16_half(thr);
-                t2 = hv | (hv << 16);
+                const uint32_t t2 = hv | (hv << 16);
+                uint64_t cand = 0;  // images equal to T (phase B candidates)
+#pragma unroll
+                for (int j = 0; j < kPairs; ++j) {
+                    take |= pair_bits(exact ? h2_set_ge(h[j], t2) : h2_set_gt(h[j], t2)) << (2 * j);
+                    cand |= pair_bits(h2_set_eq(h[j], t2)) << (2 * j);
+                }
                 if (!exact) {
-                    mode = 1;
-                    int gt = 0;
-#pragma unroll
-                    for (int j = 0; j < kPairs; ++j) {
-                        const uint32_t g = h2_set_gt(h[j], t2);
-                        gt += ((g & 0xFFFFu) != 0u) + ((g >> 16) != 0u);
-                    }
-                    const int need = allowed - int(__reduce_add_sync(0xffffffffu, uint32_t(gt)));
-                    // the candidates (image == T) in ascending column order; the first 32 are listed
-                    int n_cand = 0;
-#pragma unroll
-                    for (int j = 0; j < kPairs; ++j) {
-                        const uint32_t e = h2_set_eq(h[j], t2);
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const bool eq = u ? (e >> 16) != 0u : (e & 0xFFFFu) != 0u;
-                            const unsigned bal = __ballot_sync(0xffffffffu, eq);
-                            const int at = n_cand + __popc(bal & lower);
-                            if (eq && at < 32) cand_col[wib][at] = (2 * j + u) * 32 + lane;
-                            n_cand += __popc(bal);
-                        }
-                    }
-                    __syncwarp();
+                    const int need = allowed - int(__reduce_add_sync(0xffffffffu, uint32_t(__popcll(take))));
+                    const int n_cand = int(__reduce_add_sync(0xffffffffu, uint32_t(__popcll(cand))));
                     if (n_cand <= 32) {
-                        // lane j ranks candidate j by its exact key (ties: the lower column, i.e. the lower j)
+                        // list the candidates in ascending column order, lane j ranks the j-th
+                        keep_mask[wib][lane] = 0;
+                        int at = 0;
+                        const unsigned any_lo = __reduce_or_sync(0xffffffffu, uint32_t(cand));
+                        const unsigned any_hi = __reduce_or_sync(0xffffffffu, uint32_t(cand >> 32));
+                        uint64_t slots = (uint64_t(any_hi) << 32) | any_lo;  // slots where some lane has one
+                        while (slots) {
+                            const int i = __ffsll(static_cast<long long>(slots)) - 1;
+                            slots &= slots - 1;
+                            const bool is_c = (cand >> i) & 1u;
+                            const unsigned bal = __ballot_sync(0xffffffffu, is_c);
+                            if (is_c) cand_col[wib][at + __popc(bal & lower)] = i * 32 + lane;
+                            at += __popc(bal);
+                        }
+                        __syncwarp();
                         uint32_t key = 0;
+                        int c = 0;
                         if (lane < n_cand) {
-                            const int c = cand_col[wib][lane];
+                            c = cand_col[wib][lane];
                             key = c == row ? kKeyPos : order_key(__ldg(srow + c));
                         }
                         int rank = 0;
@@ -580,43 +547,33 @@ __global__ void __launch_bounds__(32 * kRowsWarps) select_rows_kernel(const Sele
                             const uint32_t ki = __shfl_sync(0xffffffffu, key, i);
                             rank += (ki > key) || (ki == key && i < lane);
                         }
-                        keep_bits = __ballot_sync(0xffffffffu, lane < n_cand && rank < need);
+                        if (lane < n_cand && rank < need)
+                            atomicOr(reinterpret_cast<unsigned long long*>(&keep_mask[wib][c & 31]), 1ull << (c >> 5));
+                        __syncwarp();
+                        take |= keep_mask[wib][lane];
+                        __syncwarp();  // cand_col and keep_mask are rewritten by the next block
                     } else {
-                        wide = true;
-                        wide_keep = select_wide_candidates<kPer>(a, srow, row, start, stop, okbits, t2, need);
+                        take |= select_wide_candidates(srow, row, cand, kPer, need);
                     }
-                    __syncwarp();  // cand_col is rewritten by the next block or row
-                }
-            }
-            // output: ascending columns
-            int cbase = 0;
-#pragma unroll
-            for (int j = 0; j < kPairs; ++j) {
-                const uint32_t ge = h2_set_ge(h[j], t2);
-                const uint32_t gt = mode ? h2_set_gt(h[j], t2) : ge;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int i = 2 * j + u;
-                    const bool is_ge = u ? (ge >> 16) != 0u : (ge & 0xFFFFu) != 0u;
-                    const bool is_gt = u ? (gt >> 16) != 0u : (gt & 0xFFFFu) != 0u;
-                    bool take = is_gt;
-                    if (mode) {
-                        const bool eq = is_ge && !is_gt;
-                        const unsigned eb = __ballot_sync(0xffffffffu, eq);
-                        const int ci = cbase + __popc(eb & lower);
-                        cbase += __popc(eb);
-                        if (eq) take = wide ? ((wide_keep >> i) & 1u) != 0u : ((keep_bits >> ci) & 1u) != 0u;
-                    }
-                    const unsigned bal = __ballot_sync(0xffffffffu, take);
-                    if (take) out[pos + __popc(bal & lower)] = i * 32 + lane;
-                    pos += __popc(bal);
                 }
             }
         }
-        const int* glob = a.ok_list + (a.n_kv_ok - a.n_global_ok);
-        for (int i = lane; i < a.n_global_ok; i += 32) out[pos + i] = __ldg(glob + i);
-        if (lane == 0) a.kept_cnt[rowid] = pos + a.n_global_ok;
+        // output: ascending columns, over the slots where some lane keeps a column
+        const unsigned any_lo = __reduce_or_sync(0xffffffffu, uint32_t(take));
+        const unsigned any_hi = __reduce_or_sync(0xffffffffu, uint32_t(take >> 32));
+        uint64_t slots = (uint64_t(any_hi) << 32) | any_lo;
+        while (slots) {
+            const int i = __ffsll(static_cast<long long>(slots)) - 1;
+            slots &= slots - 1;
+            const bool t = (take >> i) & 1u;
+            const unsigned bal = __ballot_sync(0xffffffffu, t);
+            if (t) out[pos + __popc(bal & lower)] = i * 32 + lane;
+            pos += __popc(bal);
+        }
     }
+    const int* glob = a.ok_list + (a.n_kv_ok - a.n_global_ok);
+    for (int i = lane; i < a.n_global_ok; i += 32) out[pos + i] = __ldg(glob + i);
+    if (lane == 0) a.kept_cnt[rowid] = pos + a.n_global_ok;
 }
 
 }  // namespace veda

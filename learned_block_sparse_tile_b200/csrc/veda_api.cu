@@ -408,28 +408,36 @@ extern "C" int veda_score(const veda_layout* layout, const float* feats_q, const
     return launch_check("gemm_f32_kernel");
 }
 
-template <int kPer, bool kPrefetch>
-static int launch_rows(DeviceState* ds, const SelectArgs& a, int64_t n_rows, cudaStream_t st) {
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_rows_kernel<kPer, kPrefetch>,
-                                                                  32 * kRowsWarps, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor(select_rows_kernel)");
-    const int64_t want = (n_rows + kRowsWarps - 1) / kRowsWarps;
-    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(ds->sms) * std::max(per_sm, 1))));
-    select_rows_kernel<kPer, kPrefetch><<<grid, 32 * kRowsWarps, 0, st>>>(a);
+template <int kPer>
+static int launch_rows(const SelectArgs& a, int64_t n_rows, cudaStream_t st) {
+    const int64_t grid = (n_rows + kRowsWarps - 1) / kRowsWarps;
+    if (grid > 0x7fffffff) return fail(VEDA_ERR_UNSUPPORTED, "veda_select: too many rows for one launch");
+    if (a.n_blocks == 2)
+        select_rows_kernel<kPer, true><<<unsigned(grid), 32 * kRowsWarps, 0, st>>>(a);
+    else
+        select_rows_kernel<kPer, false><<<unsigned(grid), 32 * kRowsWarps, 0, st>>>(a);
     return launch_check("select_rows_kernel");
 }
 
-static int launch_select_rows(DeviceState* ds, int per, const SelectArgs& a, int64_t n_rows, cudaStream_t st) {
+// One warp per row; kPer = slots per lane, the row's width / 32 rounded up to a multiple of 4.
+static int launch_select_rows(int per, const SelectArgs& a, int64_t n_rows, cudaStream_t st) {
     switch (per) {
-        case 8: return launch_rows<8, true>(ds, a, n_rows, st);
-        case 16: return launch_rows<16, true>(ds, a, n_rows, st);
-        case 24: return launch_rows<24, true>(ds, a, n_rows, st);
-        case 32: return launch_rows<32, true>(ds, a, n_rows, st);
-        case 40: return launch_rows<40, false>(ds, a, n_rows, st);
-        case 48: return launch_rows<48, false>(ds, a, n_rows, st);
-        case 56: return launch_rows<56, false>(ds, a, n_rows, st);
-        default: return launch_rows<64, false>(ds, a, n_rows, st);
+        case 4: return launch_rows<4>(a, n_rows, st);
+        case 8: return launch_rows<8>(a, n_rows, st);
+        case 12: return launch_rows<12>(a, n_rows, st);
+        case 16: return launch_rows<16>(a, n_rows, st);
+        case 20: return launch_rows<20>(a, n_rows, st);
+        case 24: return launch_rows<24>(a, n_rows, st);
+        case 28: return launch_rows<28>(a, n_rows, st);
+        case 32: return launch_rows<32>(a, n_rows, st);
+        case 36: return launch_rows<36>(a, n_rows, st);
+        case 40: return launch_rows<40>(a, n_rows, st);
+        case 44: return launch_rows<44>(a, n_rows, st);
+        case 48: return launch_rows<48>(a, n_rows, st);
+        case 52: return launch_rows<52>(a, n_rows, st);
+        case 56: return launch_rows<56>(a, n_rows, st);
+        case 60: return launch_rows<60>(a, n_rows, st);
+        default: return launch_rows<64>(a, n_rows, st);
     }
 }
 
@@ -469,9 +477,9 @@ extern "C" int veda_select(const veda_layout* layout, const float* scores, int32
     for (int c = 0; c < d.n_video; ++c) a.all_ok &= layout->valid_count[c] > 0;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d.n_video <= 32 * 64) {
-        // persistent warps, one row at a time (rows of up to 2048 video tiles)
-        const int per = ((d.n_video + 31) / 32 + 7) / 8 * 8;  // slots per lane, a multiple of 8
-        return launch_select_rows(ds, per, a, int64_t(n_heads) * d.n_video, st);
+        // one warp per row (rows of up to 2048 video tiles)
+        const int per = ((d.n_video + 31) / 32 + 3) / 4 * 4;  // slots per lane, a multiple of 4
+        return launch_select_rows(per, a, int64_t(n_heads) * d.n_video, st);
     }
     if (widest <= 32 * 64) {
         // one warp per row, the block's keys in registers

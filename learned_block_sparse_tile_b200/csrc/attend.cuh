@@ -6,12 +6,12 @@
 // real rows are a prefix, so slot j of tile t is live iff j < valid_count[t]); a row that sees no key
 // gives 0. Then "tiles", scatter_: each real query slot goes to its packed row of the output.
 //
-// Design: one persistent CTA per SM, 384 threads, work items = (head, query tile), one item at a time.
-// The item's kept key tiles are split between two softmax warpgroups by parity, each with its own online
+// Design: one persistent CTA per SM, 640 threads, work items = (head, query tile), one item at a time.
+// The item's kept key tiles are split between two softmax groups by parity, each with its own online
 // softmax state and its own O accumulator in TMEM; the two partial results are merged at the end of the
 // item. While one group computes its softmax the tensor core works on the other group's tiles.
-//   warp 0       TMA producer of Q (one buffer) and K (ring of 3); warp 2: TMA producer of V (ring of 3).
-//                Every box is 128 rows x 128 bytes with the 128-byte swizzle.
+//   warp 0       TMA producer of Q (one buffer) and K (ring); warp 2: TMA producer of V (ring). Every box
+//                is 128 rows x 128 bytes with the 128-byte swizzle.
 //   warp 1       TMEM owner and MMA issuer: the whole warp runs the issue loop (its waits, descriptors and
 //                ring positions are warp-uniform) and elect.sync lets one lane issue each tcgen05 instruction,
 //                which keeps the issuer's instruction count low next to the softmax warps sharing its
@@ -19,13 +19,19 @@
 //                the S columns of group j%2, then O_(j%2) += P_j V_j with P read from TMEM where the group
 //                left it (the "TS" form) and V from shared memory. Issue order per item: S_0, S_1, then per
 //                tile PV_j followed by S_(j+2).
-//   warps 4-7    softmax group 0 (tiles 0, 2, 4, ...); warps 8-11 group 1 (tiles 1, 3, 5, ...). One thread
-//                per query row (its TMEM lane): masks key slots past the tile's real rows, keeps a running
-//                max (O is rescaled only when the max grows by more than 2^8, which bounds P by 256), and
-//                writes P as bf16 over its S columns. exp2 runs partly on the MUFU and partly as a polynomial
-//                on the FMA pipe. At the end of the item the groups exchange (max, sum) per row and each
-//                writes half of the output columns: (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / sum.
-// TMEM columns: S/P of group 0 [0,128), group 1 [128,256); O of group 0 [256, 256 + D), group 1 [384, 384 + D).
+//   warps 4-11   softmax group 0 (tiles 0, 2, 4, ...); warps 12-19 group 1 (tiles 1, 3, 5, ...). Each query
+//                row (its TMEM lane) has two threads in its group, in warps four apart: one takes key
+//                columns 0-63 of each S tile, the other 64-127, so a tile's softmax is split over eight
+//                warps. Each masks key slots past the tile's real rows, exponentiates its half against the
+//                row's running reference m (O is rescaled only when the max grows by more than 2^8, which
+//                bounds P by 256; with the logit bound, an item's later tiles keep the first tile's m), and
+//                writes P as bf16 over its own S columns. The two halves of a row exchange partial maxima
+//                whenever a tile takes the row max. exp2 runs partly on the MUFU and partly as a polynomial
+//                on the FMA pipe. At the end of the item the four threads of a row exchange (max, sum)
+//                and each writes a quarter of the output columns:
+//                (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / sum.
+// TMEM columns: S of group 0 [0,128), group 1 [128,256), P of a group over its S columns [0,32) (keys 0-63)
+// and [64,96) (keys 64-127); O of group 0 [256, 256 + D), group 1 [384, 384 + D).
 // Loads (kDirect): the tile-order variant reads head-major tile copies through 2D maps (tile t of head h
 // at rows (h N + 128 t) of [H' N, D]). The gather-free variant reads the packed [S, H, D] tensors: a span
 // tile is one 5D box (st, sh, sw, 1, 64) of its span's grid at the tile's origin, a global tile one 3D box
@@ -115,19 +121,22 @@ struct AttendCfg {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static constexpr bool kFp8 = kQK != kQKBf16;  // Q and K are 8-bit codes (1 byte per element)
     static_assert(!kFp8 || D == 128, "the 8-bit Q/K variants are built for head_dim 128");
-    static constexpr int kWarps = 12;
+    static constexpr int kWarps = 20;  // copy/MMA warpgroup (warps 0-3) + two softmax groups of eight warps
     static constexpr int kThreads = 32 * kWarps;
     static constexpr int kQKBytes = 128 * D * (kFp8 ? 1 : 2);  // one Q or K tile
     static constexpr int kTileBytes = 128 * D * 2;             // one V tile (bf16)
     static constexpr int kBoxesQK = kFp8 ? 1 : D / 64;         // 128-byte-wide TMA boxes per Q/K tile
     static constexpr int kBoxes = D / 64;                      // 64-column (128-byte) TMA boxes per V tile
-    static constexpr int kKStages = kFp8 ? 4 : 3;              // K ring depth
-    static constexpr int kVStages = kFp8 ? 4 : 3;              // V ring depth
-    // header (barriers, then the [2 groups][128 rows] (max, sum) exchange) first, then the 1024-aligned
-    // tiles; with a 1024-aligned dynamic base this fills the 227 KB a CTA may use at head_dim 128
+    static constexpr int kKStages = kFp8 ? 4 : (D == 128 ? 2 : 3);  // K ring depth
+    static constexpr int kVStages = kFp8 ? 4 : 3;                    // V ring depth
+    // header first: barriers; the end-of-item (max, partial sum) of each [group][half][row]; the
+    // [parity][group][half][row] partial row maxima the two halves of a row exchange. Then the 1024-aligned
+    // tiles (at head_dim 128: 201 KB of the 227 KB a CTA may use)
     static constexpr int kOffBar = 0;
-    static constexpr int kOffStats = 256;
-    static constexpr int kHeader = 3072;
+    static constexpr int kOffStats = 512;
+    static constexpr int kOffXch = kOffStats + 2 * 2 * 128 * 8;
+    static constexpr int kHeader = 9216;
+    static_assert(kOffXch + 2 * 2 * 2 * 128 * 4 <= kHeader, "header layout");
     static constexpr int kOffQ = kHeader;
     static constexpr int kOffK = kOffQ + kQKBytes;
     static constexpr int kOffV = kOffK + kKStages * kQKBytes;
@@ -144,6 +153,7 @@ struct AttendBars {
     uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2], o_done[2];
     uint64_t o_empty, merge, drain;
+    uint64_t pair[2][4];  // per group and TMEM lane quarter: the two halves' row-max exchange
 };
 
 // Number of kept tiles of an item and its list. Warp-collective (all 32 lanes, same result in each).
@@ -209,7 +219,7 @@ struct GroupId {
 __device__ __forceinline__ int group_tiles(int n, int w) { return (n - w + 1) >> 1; }
 
 template <int D, int kQK, bool kDirect>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
     attend_kernel(const __grid_constant__ AttendMaps maps, const AttendArgs a) {
     using C = AttendCfg<D, kQK>;
     constexpr bool kFp8 = C::kFp8;  // 8-bit Q/K codes (either format)
@@ -223,7 +233,7 @@ __global__ void __launch_bounds__(384, 1)
     AttendBars& B = *reinterpret_cast<AttendBars*>(smem + C::kOffBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&B + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float2* stats = reinterpret_cast<float2*>(smem + C::kOffStats);  // [2 groups][128 rows] (max, sum)
+    float2* stats = reinterpret_cast<float2*>(smem + C::kOffStats);  // [2 groups][2 halves][128 rows] (max, sum)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -239,11 +249,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int w = 0; w < 2; ++w) {
             ptx::mbar_init(&B.s_full[w], 1);
-            ptx::mbar_init(&B.p_full[w], 128);
+            ptx::mbar_init(&B.p_full[w], 256);
             ptx::mbar_init(&B.o_done[w], 1);
+            for (int q = 0; q < 4; ++q) ptx::mbar_init(&B.pair[w][q], 64);
         }
-        ptx::mbar_init(&B.o_empty, 256);
-        ptx::mbar_init(&B.merge, 256);
+        ptx::mbar_init(&B.o_empty, 512);
+        ptx::mbar_init(&B.merge, 512);
         ptx::mbar_init(&B.drain, 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
@@ -264,12 +275,12 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = a.timeout_ns;
 
-    // registers: the copy/MMA warpgroup (warps 0-3) hands most of its share to the two softmax warpgroups,
-    // whose 128-column rows of S then fit without spilling. Each role sets its budget at the top of its
-    // own branch (the compiler allocates each branch within it); the budgets add up to exactly the
-    // 384 x 168 registers the block is launched with, so the increases can always be granted.
-    constexpr uint32_t kRegsLow = 56, kRegsHigh = 224;
-    static_assert(128 * kRegsLow + 256 * kRegsHigh == 384 * 168, "register split");
+    // registers: the copy/MMA warpgroup (warps 0-3) hands most of its share to the four softmax warpgroups,
+    // whose 64-column halves of S then fit. Each role sets its budget at the top of its own branch (the
+    // compiler allocates each branch within it); the budgets add up to no more than the 640 x 96 registers
+    // the block is launched with, so the increases can always be granted.
+    constexpr uint32_t kRegsLow = 56, kRegsHigh = 104;
+    static_assert(128 * kRegsLow + 512 * kRegsHigh <= 640 * 96, "register split");
     if (warp == 3) {
         ptx::regs_dec<kRegsLow>();  // idle, but part of the copy/MMA warpgroup
     } else if (warp == 0 || warp == 2) {
@@ -403,9 +414,10 @@ __global__ void __launch_bounds__(384, 1)
                         const uint64_t dvs = dv + uint64_t(vs * (C::kTileBytes >> 4));
                         const uint32_t o = tmem + 256 + 128 * w, p = tmem + 128 * w;
 #pragma unroll
+                        // P of keys 0-63 sits in the group's columns 0-31, of keys 64-127 in 64-95
                         for (int kk = 0; kk < 8; ++kk)
-                            ptx::mma_bf16_ts_w(o, p + kk * 8, dvs + uint64_t(kk * (2048 >> 4)), C::kIdescPV,
-                                               (jj >= 2 || kk > 0) ? 1u : 0u);
+                            ptx::mma_bf16_ts_w(o, p + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+                                               dvs + uint64_t(kk * (2048 >> 4)), C::kIdescPV, (jj >= 2 || kk > 0) ? 1u : 0u);
                         ptx::mma_commit_w(&B.v_empty[vs]);
                         if (jj >= n - 2) ptx::mma_commit_w(&B.o_done[w]);  // the group's last tile of the item
                         if (++vs == VS) vs = 0, vph ^= 1;
@@ -457,18 +469,40 @@ __global__ void __launch_bounds__(384, 1)
         }
     } else if (warp >= 4) {
         ptx::regs_inc<kRegsHigh>();
-        // ------------------------------------------------------------- softmax groups (warps 4-7, 8-11)
-        const int w = (warp - 4) >> 2;  // group: item-local tiles j with j % 2 == w
-        const int q4 = warp & 3;        // TMEM lane quarter this warp may access
+        // ------------------------------------------------------------- softmax groups (warps 4-11, 12-19)
+        // Group w takes the item-local tiles j with j % 2 == w. Each query row (its TMEM lane) is shared by
+        // two threads of the group, in warps four apart (the same lane quarter): half 0 takes key columns
+        // 0-63 of every S tile, half 1 columns 64-127, and each writes its P (bf16 pairs) over the first 32
+        // of its own S columns, so neither overwrites S the other has yet to read. The two halves keep one
+        // reference m per row: they exchange partial row maxima (through shared memory and a bounded
+        // per-pair barrier) on tiles that take the row max - with the logit bound only an item's first.
+        const int sw = warp - 4;
+        const int w = sw >> 3;           // group
+        const int half = (sw >> 2) & 1;  // key columns [64 half, 64 half + 64) of each S tile
+        const int q4 = warp & 3;         // TMEM lane quarter this warp may access
         const int row = q4 * 32 + lane;
         const uint32_t lane_base = uint32_t(q4 * 32) << 16;
-        const uint32_t t_s = tmem + lane_base + 128 * w;        // S / P of this group
-        const uint32_t t_o = tmem + lane_base + 256 + 128 * w;  // O of this group
+        const uint32_t t_s = tmem + lane_base + 128 * w + 64 * half;  // this half's S columns (its P: the first 32)
+        const uint32_t t_o = tmem + lane_base + 256 + 128 * w;        // O of this group
         const uint32_t t_o0 = tmem + lane_base + 256;
+        float* xch = reinterpret_cast<float*>(smem + C::kOffXch);      // [parity][group][half][row]
+        uint64_t* pair_bar = &B.pair[w][q4];
+        int xc = 0;  // row-max exchanges so far: the pair barrier's phase and the exchange buffer's parity
+        // this thread's partial row max -> the row max of both halves (false: a wait gave up)
+        auto pair_max = [&](float pm, float* mx) -> bool {
+            float* x = xch + ((xc & 1) * 4 + w * 2) * 128;
+            x[half * 128 + row] = pm;
+            ptx::mbar_arrive(pair_bar);  // release: the store above is visible once the phase completes
+            const bool done = ptx::mbar_wait(pair_bar, xc & 1, abort_flag, tmo);
+            ++xc;
+            *mx = fmaxf(pm, x[(half ^ 1) * 128 + row]);
+            return done;
+        };
         int cu = 0;          // tiles this group has had so far (barrier phases)
         int it = 0, t = 0;   // items with tiles so far; tiles so far (K ring positions)
         int od_mine = 0, od_other = 0;  // o_done phases of this group and the other: one per item with a tile
-        const bool releaser = (warp & 3) == 0 && lane == 0;  // one thread per group frees K slots
+        const bool releaser = (sw & 7) == 0 && lane == 0;  // one thread per group frees K slots
+        constexpr int kCols = D / 4;  // output columns each thread writes (four threads per row)
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
@@ -479,19 +513,21 @@ __global__ void __launch_bounds__(384, 1)
             const bool head_ok = head >= 0 && head < a.h_total;
             if (!head_ok && threadIdx.x == 128) atomicOr(a.err, 4);
             const int prow = head_ok ? __ldg(a.perm + int64_t(qt) * 128 + row) : -1;
-            // this group writes output columns [w D/2, (w + 1) D/2) of its rows
+            // this thread writes output columns [(2 w + half) D / 4, (2 w + half + 1) D / 4) of its row
+            const int ocol = (2 * w + half) * kCols;
             __nv_bfloat16* dst = a.out + int64_t(prow < 0 ? 0 : prow) * a.out_s0 +
-                                 int64_t(head_ok ? head : 0) * a.out_s1 + w * (D / 2);
+                                 int64_t(head_ok ? head : 0) * a.out_s1 + ocol;
             if (n == 0) {
                 if (prow >= 0) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int c = 0; c < D / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
+                    for (int c = 0; c < kCols / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
                 }
                 continue;
             }
             const int nw = group_tiles(n, w);
-            // log2-domain bound on every logit of this row (padding slots need none)
+            // log2-domain bound on every logit of this row (padding slots need none); both halves of a row
+            // compute the same value
             float bound = INFINITY;
             if (!kFp8 && a.q_row_sq != nullptr && prow >= 0)
                 bound = sqrtf(__ldg(a.q_row_sq + int64_t(hh) * a.seq_len + prow) * __ldg(a.k_max_sq + hh)) *
@@ -524,17 +560,16 @@ __global__ void __launch_bounds__(384, 1)
                 // issued after the PV of the group's previous tile, so that PV is complete as well: O may be
                 // rescaled and the P columns rewritten without another wait.
                 if (releaser) ptx::mbar_arrive(&B.k_empty[(t + 2 * k + w) % KS]);
-                uint32_t s[128];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    ptx::tmem_ld32(t_s + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(s + 32 * i));
+                uint32_t s[64];
+                ptx::tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
+                ptx::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
                 ptx::tmem_wait_ld();
                 if constexpr (kQK == kQKI8) {
                     // int32 -> fp32, exactly: adding the bit pattern of 1.5 * 2^23 puts |S| < 2^22 in the
                     // low mantissa bits of a float in [2^23, 2^24); subtracting 1.5 * 2^23 is then exact
                     const uint64_t magic = ptx::f2_pack(-12582912.f, -12582912.f);
 #pragma unroll
-                    for (int c = 0; c < 128; c += 2) {
+                    for (int c = 0; c < 64; c += 2) {
                         float f0, f1;
                         ptx::f2_unpack(ptx::f2_add(ptx::f2_pack(__uint_as_float(s[c] + 0x4B400000u),
                                                                 __uint_as_float(s[c + 1] + 0x4B400000u)), magic), f0, f1);
@@ -546,31 +581,34 @@ __global__ void __launch_bounds__(384, 1)
                     if constexpr (kDirect) {
                         // box order: the tile's rows sit where its mask says (padding in place)
                         const uint4 m = __ldg(a.tile_mask + __shfl_sync(0xffffffffu, my_tile, k & 31));
-                        const uint32_t mw[4] = {m.x, m.y, m.z, m.w};
+                        const uint32_t mw0 = half ? m.z : m.x, mw1 = half ? m.w : m.y;
 #pragma unroll
-                        for (int c = 0; c < 128; ++c)
-                            if (((mw[c >> 5] >> (c & 31)) & 1u) == 0) s[c] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 64; ++c)
+                            if ((((c < 32 ? mw0 : mw1) >> (c & 31)) & 1u) == 0) s[c] = __float_as_uint(-INFINITY);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 128; ++c)
-                            if (c >= vc) s[c] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 64; ++c)
+                            if (64 * half + c >= vc) s[c] = __float_as_uint(-INFINITY);
                     }
                 }
                 bool resc = false;
                 float alpha = 1.f;
                 if (!skip) {
-                    // row max: 8 independent chains of 3-input maxima
+                    // row max: 8 independent chains of 3-input maxima over this half, then both halves
                     float mx8[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(__uint_as_float(s[q]), __uint_as_float(s[8 + q]));
 #pragma unroll
-                    for (int c = 16; c < 128; c += 16) {
+                    for (int c = 16; c < 64; c += 16) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             mx8[q] = ptx::max3(mx8[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
                     }
-                    const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
-                                               fmaxf(mx8[6], mx8[7]));
+                    const float pmx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
+                                                fmaxf(mx8[6], mx8[7]));
+                    float mx;
+                    ok = pair_max(pmx, &mx);
+                    if (!ok) break;
                     const float m_new = mx * sl2;
                     resc = m_new > m_ref + 8.0f;
                     if (resc) {
@@ -578,6 +616,7 @@ __global__ void __launch_bounds__(384, 1)
                         lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
                         m_ref = m_new;
                     }
+                    // the same decision in both warps of the pair: bound and m_ref are equal for a row
                     if (k == 0 && a.q_row_sq != nullptr)
                         skip = __all_sync(0xffffffffu, prow < 0 || bound - m_ref <= kSkipLimit);
                 }
@@ -586,7 +625,7 @@ __global__ void __launch_bounds__(384, 1)
                 uint64_t acc[4] = {ptx::f2_pack(0.f, 0.f), ptx::f2_pack(0.f, 0.f), ptx::f2_pack(0.f, 0.f),
                                    ptx::f2_pack(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < 128; c += 2) {
+                for (int c = 0; c < 64; c += 2) {
                     const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2, negm2);
                     float p0, p1;
                     if (((c >> 1) & 7) < kPolyPairs) {  // this pair on the FMA pipe
@@ -601,23 +640,27 @@ __global__ void __launch_bounds__(384, 1)
                     s[c >> 1] = ptx::pack_bf16(p0, p1);
                 }
                 lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])));
+                // P (bf16 pairs of this half's 64 keys) over the first 32 of its S columns: the A operand
+                // of O += P V reads keys 0-63 from the group's columns 0-31 and keys 64-127 from 64-95
+                ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
+                ptx::tmem_wait_st();
                 if (k > 0) {
+                    // a new reference: rescale this half's share of the accumulator's columns before P is
+                    // handed over (P is stored first, so its registers are free here)
                     if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
-                        for (int i = 0; i < D / 32; ++i) {
+#pragma unroll 1
+                        for (int i = 0; i < D / 64; ++i) {
                             uint32_t o[32];
-                            ptx::tmem_ld32(t_o + 32 * i, o);
+                            const uint32_t ta = t_o + (D / 2) * half + 32 * i;
+                            ptx::tmem_ld32(ta, o);
                             ptx::tmem_wait_ld();
 #pragma unroll
                             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                            ptx::tmem_st32(t_o + 32 * i, o);
+                            ptx::tmem_st32(ta, o);
                         }
+                        ptx::tmem_wait_st();
                     }
                 }
-                // P (bf16 pairs) over the first 64 S columns: the A operand of O += P V
-                ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
-                ptx::tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
-                ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&B.p_full[w]);
             }
@@ -635,34 +678,34 @@ __global__ void __launch_bounds__(384, 1)
             cu += nmine;
             t += n;
             if (!ok) break;
-            // merge the two groups: exchange (max, sum) per row through shared memory
+            // merge the two groups: each half publishes its group's reference and its part of the row sum
             float l0, l1;
             ptx::f2_unpack(lsum, l0, l1);
-            stats[w * 128 + row] = make_float2(m_ref, l0 + l1);
+            stats[(w * 2 + half) * 128 + row] = make_float2(m_ref, l0 + l1);
             ptx::mbar_arrive(&B.merge);
             ok = ptx::mbar_wait(&B.merge, it & 1, abort_flag, tmo);
             ++it;
             if (!ok) break;
-            const float2 st0 = stats[row], st1 = stats[128 + row];
-            const float m = fmaxf(st0.x, st1.x);
-            const float a0 = st0.y > 0.f ? ptx::ex2(st0.x - m) : 0.f;
-            const float a1 = st1.y > 0.f ? ptx::ex2(st1.x - m) : 0.f;
-            const float den = a0 * st0.y + a1 * st1.y;
+            const float2 g00 = stats[row], g01 = stats[128 + row], g10 = stats[256 + row], g11 = stats[384 + row];
+            const float m0 = g00.x, sum0 = g00.y + g01.y, m1 = g10.x, sum1 = g10.y + g11.y;
+            const float m = fmaxf(m0, m1);
+            const float a0 = sum0 > 0.f ? ptx::ex2(m0 - m) : 0.f;
+            const float a1 = sum1 > 0.f ? ptx::ex2(m1 - m) : 0.f;
+            const float den = a0 * sum0 + a1 * sum1;
             const float inv = den > 0.f ? 1.f / den : 0.f;
             const float s0 = a0 * inv, s1 = a1 * inv;
             ptx::tc_fence_after();
-            // both accumulators' columns of our half are read (and merged into bf16 pairs) before O is
-            // released to the next item's first PV; the global stores come after the release
-            uint32_t res[D / 4];
+            // both accumulators' columns of this thread's share are read (and merged into bf16 pairs) before
+            // O is released to the next item's first PV; the global stores come after the release
+            uint32_t res[kCols / 2];
 #pragma unroll
-            for (int i = 0; i < D / 64; ++i) {
-                const uint32_t col = w * (D / 2) + 32 * i;
-                uint32_t o0[32], o1[32];
-                ptx::tmem_ld32(t_o0 + col, o0);
-                ptx::tmem_ld32(t_o0 + 128 + col, o1);
+            for (int h16 = 0; h16 < kCols / 16; ++h16) {  // 16 columns at a time (keeps registers for P's loop)
+                uint32_t o0[16], o1[16];
+                ptx::tmem_ld16(t_o0 + ocol + 16 * h16, o0);
+                ptx::tmem_ld16(t_o0 + 128 + ocol + 16 * h16, o1);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     float v[2];
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
@@ -670,7 +713,7 @@ __global__ void __launch_bounds__(384, 1)
                         const float x1 = s1 != 0.f ? __uint_as_float(o1[2 * c + u]) * s1 : 0.f;
                         v[u] = x0 + x1;
                     }
-                    res[16 * i + c] = ptx::pack_bf16(v[0], v[1]);
+                    res[8 * h16 + c] = ptx::pack_bf16(v[0], v[1]);
                 }
             }
             ptx::tc_fence_before();
@@ -678,7 +721,7 @@ __global__ void __launch_bounds__(384, 1)
             if (prow >= 0) {
                 uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-                for (int c = 0; c < D / 16; ++c) d4[c] = make_uint4(res[4 * c], res[4 * c + 1], res[4 * c + 2], res[4 * c + 3]);
+                for (int c = 0; c < kCols / 8; ++c) d4[c] = make_uint4(res[4 * c], res[4 * c + 1], res[4 * c + 2], res[4 * c + 3]);
             }
         }
     }

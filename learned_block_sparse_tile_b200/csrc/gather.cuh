@@ -14,6 +14,7 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
 #include "quant.cuh"
 
 namespace veda {
@@ -58,40 +59,63 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
     const __nv_bfloat16* src = a.x + head * a.s1 + c * 8;
 
     uint4 v[kPasses];
+    int pr[kPasses];  // packed row of each pass's row (-1: padding)
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
         const int r = r0 + p * kRpp;
-        const int pr = __ldg(a.perm + int64_t(tile) * 128 + r);
-        v[p] = pr >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + int64_t(pr) * a.s0)) : make_uint4(0, 0, 0, 0);
+        pr[p] = __ldg(a.perm + int64_t(tile) * 128 + r);
+        v[p] = pr[p] >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + int64_t(pr[p]) * a.s0)) : make_uint4(0, 0, 0, 0);
     }
     if (a.row_sq != nullptr || a.max_sq != nullptr) {
-        // ||x||^2 per row: each thread squares its 8 columns, the kTpr threads of a row add up
-        __shared__ unsigned cta_max;
-        if (tid == 0) cta_max = 0u;
-        __syncthreads();
-        float best = 0.f;
+        // ||x||^2 per row. Each thread squares its 8 columns of each of its kPasses rows; the kTpr threads
+        // of a row then add up with a transposed butterfly: at every step a thread keeps half of its rows
+        // and hands the other half to its partner, so the kPasses rows cost kPasses - 1 + log2(kTpr /
+        // kPasses) shuffles (when kTpr >= kPasses) instead of kPasses log2(kTpr)
+        static_assert(kTpr >= kPasses, "one row per thread pair after the butterfly");
+        float ss[kPasses];
 #pragma unroll
         for (int p = 0; p < kPasses; ++p) {
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[p]);
-            float ss = 0.f;
+            uint64_t acc = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(h2[e]);
-                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                const uint64_t f2 = ptx::f2_pack(f.x, f.y);
+                acc = ptx::f2_fma(f2, f2, acc);
             }
+            float lo, hi;
+            ptx::f2_unpack(acc, lo, hi);
+            ss[p] = lo + hi;
+        }
+        // after the step with distance d (kPasses / 2, ..., 1 in units of rows) a thread holds the partial
+        // sums of the rows whose index bits match its own lane bits at those positions
 #pragma unroll
-            for (int off = 1; off < kTpr; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            const int pr = __ldg(a.perm + int64_t(tile) * 128 + r0 + p * kRpp);
-            if (pr >= 0) {
-                if (a.row_sq != nullptr && c == 0) a.row_sq[int64_t(hh) * a.seq_len + pr] = ss;
-                best = fmaxf(best, ss);
+        for (int d = kPasses / 2, bit = kPasses / 2; d >= 1; d >>= 1, bit >>= 1) {
+            const bool upper = (c & bit) != 0;
+#pragma unroll
+            for (int i = 0; i < d; ++i) {
+                // keep rows i + (upper ? d : 0), send the other
+                const float send = upper ? ss[i] : ss[i + d];
+                const float got = __shfl_xor_sync(0xffffffffu, send, bit);
+                ss[i] = (upper ? ss[i + d] : ss[i]) + got;
             }
         }
-        if (a.max_sq != nullptr) {
+        // ss[0] is now the partial sum of row p = c % kPasses over the threads c' == c (mod kPasses)
 #pragma unroll
-            for (int off = kTpr; off < 32; off <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, off));
+        for (int off = kPasses; off < kTpr; off <<= 1) ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], off);
+        const int pm = c % kPasses;
+        int my_pr = pr[0];
+#pragma unroll
+        for (int p = 1; p < kPasses; ++p) my_pr = pm == p ? pr[p] : my_pr;
+        __shared__ unsigned cta_max;
+        if (tid == 0) cta_max = 0u;
+        __syncthreads();
+        if (c < kPasses && my_pr >= 0) {
+            if (a.row_sq != nullptr) a.row_sq[int64_t(hh) * a.seq_len + my_pr] = ss[0];
             // non-negative floats order as their bit patterns
-            if ((tid & 31) == 0) atomicMax(&cta_max, __float_as_uint(best));
+            if (a.max_sq != nullptr) atomicMax(&cta_max, __float_as_uint(ss[0]));
+        }
+        if (a.max_sq != nullptr) {
             __syncthreads();
             if (tid == 0) atomicMax(a.max_sq + hh, cta_max);
         }
@@ -108,12 +132,15 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
 
     if (a.feats == nullptr || tile >= a.n_video) return;
 
-    float sum[8], mx[8], mn[8];
+    // column sums in fp32 (packed pairs), maxima and minima on the bf16 pairs themselves (exact either way)
+    uint64_t sum2[4];
+    __nv_bfloat162 mx2[4], mn2[4];
+    const __nv_bfloat162 ninf = __floats2bfloat162_rn(-INFINITY, -INFINITY), pinf = __floats2bfloat162_rn(INFINITY, INFINITY);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        sum[e] = 0.f;
-        mx[e] = -INFINITY;
-        mn[e] = INFINITY;
+    for (int e = 0; e < 4; ++e) {
+        sum2[e] = ptx::f2_pack(0.f, 0.f);
+        mx2[e] = ninf;
+        mn2[e] = pinf;
     }
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
@@ -122,14 +149,21 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(h2[e]);
-                sum[2 * e] += f.x;
-                sum[2 * e + 1] += f.y;
-                mx[2 * e] = fmaxf(mx[2 * e], f.x);
-                mx[2 * e + 1] = fmaxf(mx[2 * e + 1], f.y);
-                mn[2 * e] = fminf(mn[2 * e], f.x);
-                mn[2 * e + 1] = fminf(mn[2 * e + 1], f.y);
+                sum2[e] = ptx::f2_add(sum2[e], ptx::f2_pack(f.x, f.y));
+                mx2[e] = __hmax2(mx2[e], h2[e]);
+                mn2[e] = __hmin2(mn2[e], h2[e]);
             }
         }
+    }
+    float sum[8], mx[8], mn[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        ptx::f2_unpack(sum2[e], sum[2 * e], sum[2 * e + 1]);
+        const float2 hi = __bfloat1622float2(mx2[e]), lo = __bfloat1622float2(mn2[e]);
+        mx[2 * e] = hi.x;
+        mx[2 * e + 1] = hi.y;
+        mn[2 * e] = lo.x;
+        mn[2 * e + 1] = lo.y;
     }
     // lanes that hold the same columns differ in the bits above log2(kTpr)
 #pragma unroll

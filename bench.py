@@ -50,7 +50,7 @@ def peaks():
 
 def attend_source_hash():
     h = hashlib.sha256()
-    for f in ("attend.cuh", "ptx.cuh"):
+    for f in ("attend.cuh", "attend_pair.cuh", "ptx.cuh"):
         h.update(open(os.path.join(ROOT, "learned_block_sparse_tile_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -216,7 +216,7 @@ def run_veda(args, rank, world, local):
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
                       wl.heads, wl.dim, device=f"cuda:{local}", fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk,
                       direct={"auto": None, "gathered": False, "direct": True}[args.path],
-                      logit_bound=args.logit_bound == "on")
+                      logit_bound=args.logit_bound == "on", paired=args.paired == "on")
     direct = layer.direct
     layer.set_projections(pq, pk)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
@@ -288,7 +288,10 @@ def run_veda(args, rank, world, local):
         gbs = sbytes[name] / (ms * 1e-3) / 1e9 if ms > 0 else None
         stages[name] = {"ms": round(ms, 4), "bytes": sbytes[name], "gb_s": round(gbs, 1) if gbs else None,
                         "hbm_frac": round(gbs / pk_["hbm"], 3) if gbs else None}
-    traffic = recorded_traffic(args.workload + ("/direct" if direct else ""), wl.dim)
+    traffic = recorded_traffic(args.workload + ("/direct" if direct else "") + ("/paired" if layer.paired else ""),
+                               wl.dim)
+    kernel = (f"attend_pair_kernel<{wl.dim}> (with its list merge and redo pass)" if layer.paired
+              else f"attend_kernel<{wl.dim}>")
     dense_pairs = wl.heads * (wl.seq_len / 128.0) ** 2
     res = {
         "metric": METRIC, "value": round(ms_step / world, 4), "unit": UNIT, "n_gpus": world,
@@ -301,14 +304,14 @@ def run_veda(args, rank, world, local):
                    "head_groups": [list(g["box"]) for g in layer.groups],
                    "attend_path": ("gather-free: Q/K pooled in place, tiles loaded as TMA boxes of the packed tensors"
                                    if direct else "tile-order copies of Q/K/V (gather), then attend"),
-                   "logit_bound": layer.logit_bound,
+                   "logit_bound": layer.logit_bound, "paired": layer.paired,
                    "parallelism": f"replicas x{world} (one layer per rank)",
                    "l2": "no flush: per-step inputs and outputs (2.6 GB at 104k tokens) exceed the 126 MB L2"},
         "kept_tile_tflops": round(achieved_tflops, 1),
         "kept_tile_work": work, "attended_tile_pairs": pairs,
         "work_share_of_dense": round(work / dense_pairs, 4),
         "stages": stages,
-        "roofline": {"bound": "tensor", "kernel": f"attend_kernel<{wl.dim}>", "achieved": round(achieved_tflops, 1),
+        "roofline": {"bound": "tensor", "kernel": kernel, "achieved": round(achieved_tflops, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 3),
                      "peak_kind": peak_kind, "timed_region_s": round(ms_total / 1e3, 3),
                      "frac_of_burst_peak": round(achieved_tflops / pk_["bf16"], 3),
@@ -359,6 +362,8 @@ def main():
     ap.add_argument("--logit-bound", default="on", choices=["on", "off"],
                     help="attend with the Cauchy-Schwarz logit bound (later tiles of an item may skip the row max; "
                          "the same softmax) or with the exact row max on every tile")
+    ap.add_argument("--paired", default="on", choices=["on", "off"],
+                    help="with the logit bound: the paired attend (two query tiles per work item) or the single-tile one")
     ap.add_argument("--impl", default="veda", choices=["veda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)

@@ -298,6 +298,37 @@ int veda_attend_direct(const veda_layout* layout, const void* q, const int64_t q
                        const int32_t* kept_cnt, void* out, const int64_t out_strides[3], const float* q_row_sq,
                        const float* k_max_sq, void* stream);
 
+/* Paired attend: the same operation as veda_attend / veda_attend_direct on the same lists (veda_core.py,
+ * "selection", reference_attend, then "tiles", scatter_), computed two neighbouring query tiles at a time.
+ * Video query tiles 2p and 2p + 1 of a head (and global query tiles likewise) share one CTA, which loads
+ * each key tile of the union of their two kept lists once for both, so neighbouring tiles that keep the
+ * same key tiles read them from L2 once instead of twice. Each query row takes its softmax reference
+ * from the logit bound, m = sqrt(q_row_sq * k_max_sq) D^-0.5 log2(e) - 64 (log2 units, so every 2^(s - m)
+ * is at most 2^64); no row max is taken and both softmax halves add into one accumulator per query tile.
+ * A real row whose sum of 2^(s - m) ends outside [2^-60, 2^100] (the bound loose by more than 124 log2
+ * units, or not finite) flags its query tile, and a second launch of veda_attend's kernel recomputes
+ * every row of the flagged tiles with the exact per-tile maxima. Results agree with veda_attend within
+ * rounding (sums run in another order).
+ *  q_row_sq, k_max_sq  required (device fp32, from veda_pool or veda_gather of the same Q and K).
+ *  workspace, workspace_bytes  device buffer of at least veda_attend_paired_workspace_bytes(layout,
+ *             n_heads) bytes, 256-byte aligned, owned by the caller; overwritten by the call (the merged
+ *             lists and the redo flags) and free for other use once the call's kernels have finished on
+ *             `stream`.
+ * Other arguments, limits and errors as veda_attend / veda_attend_direct (a malformed kept list is cut at
+ * its first bad entry and veda_sync_status reports VEDA_ERR_BAD_LIST); VEDA_ERR_INVALID also for NULL
+ * norms or a NULL, unaligned or too small workspace. */
+size_t veda_attend_paired_workspace_bytes(const veda_layout* layout, int32_t n_heads);
+int veda_attend_paired(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
+                       int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                       const int64_t out_strides[3], int32_t h_total, const int32_t* heads, const float* q_row_sq,
+                       const float* k_max_sq, void* workspace, size_t workspace_bytes, void* stream);
+int veda_attend_direct_paired(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
+                              const int64_t k_strides[3], const void* v, const int64_t v_strides[3], int32_t h_total,
+                              int32_t dim, const int32_t* heads, int32_t n_heads, const int32_t* kept_idx,
+                              const int32_t* kept_cnt, void* out, const int64_t out_strides[3],
+                              const float* q_row_sq, const float* k_max_sq, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* FP8 Q/K variant, step 1 (not on the pages: their kernel quantises to INT8 by a recipe they do not
  * print; this follows the FP8 e4m3 variant of the 104k budget sweep). Per (head, 128-row tile) of a
  * tile-ordered bf16 tensor: scale = amax(|x|) over the tile's real rows / 448 (1 when 0), and each code is
@@ -365,7 +396,7 @@ int veda_device_check(void);
 void veda_set_wait_timeout_ns(uint64_t ns);
 
 /* Test hook for the failure path (the pages have no counterpart): the calling thread's next veda_attend
- * withholds its Q tile loads, so the kernel's waits on them expire; the kernel then lets its in-flight
+ * (any variant; the paired ones' first kernel) withholds its Q tile loads, so the kernel's waits on them expire; the kernel then lets its in-flight
  * copies and MMAs finish, frees its tensor memory and returns, and veda_sync_status reports
  * VEDA_ERR_TIMEOUT. The output of that call is unspecified; the device stays usable. */
 void veda_debug_hold_next_attend(void);

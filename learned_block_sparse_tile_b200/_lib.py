@@ -24,6 +24,7 @@ EXPORTS = [
     "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
     "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8", "veda_layout_export_direct", "veda_pool",
     "veda_attend_direct", "veda_debug_exp2", "veda_grid_of", "veda_describe_packed_layout",
+    "veda_attend_paired_workspace_bytes", "veda_attend_paired", "veda_attend_direct_paired",
 ]
 
 VEDA_SEG_OTHER, VEDA_SEG_VIDEO, VEDA_SEG_COND, VEDA_SEG_REF_IMG = range(4)
@@ -95,6 +96,13 @@ def lib():
         L.veda_attend_direct.argtypes = [vp, p, C.POINTER(C.c_int64), p, C.POINTER(C.c_int64), p,
                                          C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, C.POINTER(C.c_int64), p,
                                          p, vp]
+        L.veda_attend_paired_workspace_bytes.argtypes = [vp, i32]
+        L.veda_attend_paired_workspace_bytes.restype = C.c_size_t
+        L.veda_attend_paired.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, p, p, p,
+                                         C.c_size_t, vp]
+        L.veda_attend_direct_paired.argtypes = [vp, p, C.POINTER(C.c_int64), p, C.POINTER(C.c_int64), p,
+                                                C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, C.POINTER(C.c_int64),
+                                                p, p, p, C.c_size_t, vp]
         L.veda_score_workspace_bytes.argtypes = [vp, i32, i32]
         L.veda_score_workspace_bytes.restype = C.c_size_t
         L.veda_score.argtypes = [vp, p, p, i32, i32, p, p, p, C.c_size_t, p, vp]
@@ -270,6 +278,37 @@ def veda_attend_direct(layout, q, k, v, kept_idx, kept_cnt, out, heads, stream=N
                                     q.shape[1], q.shape[2], _ptr(heads), heads.numel(), _ptr(kept_idx),
                                     _ptr(kept_cnt), _ptr(out), _strides(out), _ptr(q_row_sq), _ptr(k_max_sq),
                                     _stream(stream)))
+
+
+def veda_attend_paired_workspace_bytes(layout, n_heads):
+    return int(lib().veda_attend_paired_workspace_bytes(layout.handle, n_heads))
+
+
+def paired_workspace(layout, n_heads, device="cuda"):
+    """A device buffer for the paired attend of ``n_heads`` heads on ``layout`` (uint8, 256-byte aligned)."""
+    import torch
+    return torch.empty(max(veda_attend_paired_workspace_bytes(layout, n_heads), 256), dtype=torch.uint8,
+                       device=device)
+
+
+def veda_attend_paired(layout, q_t, k_t, v_t, kept_idx, kept_cnt, out, heads, q_row_sq, k_max_sq, workspace,
+                       stream=None):
+    """veda_attend two neighbouring query tiles at a time (each kept K/V tile loaded once for both), with the
+    softmax reference from the logit bound; q_row_sq / k_max_sq are required, workspace from paired_workspace."""
+    _check(lib().veda_attend_paired(layout.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), q_t.shape[0], q_t.shape[2],
+                                    _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1],
+                                    _ptr(heads), _ptr(q_row_sq), _ptr(k_max_sq), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def veda_attend_direct_paired(layout, q, k, v, kept_idx, kept_cnt, out, heads, q_row_sq, k_max_sq, workspace,
+                              stream=None):
+    """veda_attend_direct two neighbouring query tiles at a time (as veda_attend_paired)."""
+    _check(lib().veda_attend_direct_paired(layout.handle, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v),
+                                           _strides(v), q.shape[1], q.shape[2], _ptr(heads), heads.numel(),
+                                           _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), _ptr(q_row_sq),
+                                           _ptr(k_max_sq), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def veda_gather_fp8(layout, x, heads, codes, scales, feats=None, stream=None):

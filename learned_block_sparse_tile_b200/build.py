@@ -10,7 +10,8 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libveda.so")
 
 SOURCES = ["veda_api.cu", "veda_plan.cpp", "veda_score_noalloc.cu"]
-HEADERS = ["veda_internal.h", "ptx.cuh", "gather.cuh", "score.cuh", "select.cuh", "attend.cuh", "quant.cuh"]
+HEADERS = ["veda_internal.h", "ptx.cuh", "gather.cuh", "score.cuh", "select.cuh", "attend.cuh", "attend_pair.cuh",
+           "quant.cuh"]
 
 
 def nvcc_path():

@@ -92,6 +92,9 @@ struct AttendArgs {
     const float* q_row_sq;  // [n_heads, seq_len]
     const float* k_max_sq;  // [n_heads]
     int64_t seq_len;
+    // redo pass after the paired kernel (attend_pair.cuh): when set, only the query tiles (head index, tile)
+    // flagged non-zero in [n_heads, n_tiles] are processed; every other item is skipped by every role
+    const int32_t* redo_flags;
 };
 
 // With the logit bound, a softmax group takes its reference m from the exact row maxima of its first tile
@@ -194,6 +197,11 @@ __device__ __forceinline__ int item_tiles(const AttendArgs& a, int hh, int qt, c
     return n;
 }
 
+// True when a redo pass skips this query tile (see AttendArgs::redo_flags). Uniform across the CTA.
+__device__ __forceinline__ bool item_skipped(const AttendArgs& a, int hh, int qt) {
+    return a.redo_flags != nullptr && __ldg(a.redo_flags + int64_t(hh) * a.n_tiles + qt) == 0;
+}
+
 // Item order: the dense global query tiles first (they are the longest), then head-major video tiles,
 // so that neighbouring slots work on neighbouring query tiles of one head (shared K/V in L2).
 __device__ __forceinline__ void decode_item(const AttendArgs& a, int item, int* hh, int* qt) {
@@ -293,6 +301,7 @@ __global__ void __launch_bounds__(640, 1)
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
+            if (item_skipped(a, hh, qt)) continue;
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
@@ -395,6 +404,7 @@ __global__ void __launch_bounds__(640, 1)
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
+            if (item_skipped(a, hh, qt)) continue;
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
@@ -506,6 +516,7 @@ __global__ void __launch_bounds__(640, 1)
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
             int hh, qt;
             decode_item(a, item, &hh, &qt);
+            if (item_skipped(a, hh, qt)) continue;
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
@@ -622,8 +633,8 @@ __global__ void __launch_bounds__(640, 1)
                 }
                 const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
                 const uint64_t negm2 = ptx::f2_pack(negm, negm);
-                uint64_t acc[4] = {ptx::f2_pack(0.f, 0.f), ptx::f2_pack(0.f, 0.f), ptx::f2_pack(0.f, 0.f),
-                                   ptx::f2_pack(0.f, 0.f)};
+                // row sums over the bf16 P the PV product reads (eight independent chains)
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
                     const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2, negm2);
@@ -636,10 +647,11 @@ __global__ void __launch_bounds__(640, 1)
                         p0 = ptx::ex2(x0);
                         p1 = ptx::ex2(x1);
                     }
-                    acc[(c >> 1) & 3] = ptx::f2_add(acc[(c >> 1) & 3], ptx::f2_pack(p0, p1));
                     s[c >> 1] = ptx::pack_bf16(p0, p1);
+                    ptx::add_bf16x2(s[c >> 1], acc[(c >> 1) & 3], acc[4 + ((c >> 1) & 3)]);
                 }
-                lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])));
+                lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(ptx::f2_pack(acc[0], acc[4]), ptx::f2_pack(acc[1], acc[5])),
+                                                     ptx::f2_add(ptx::f2_pack(acc[2], acc[6]), ptx::f2_pack(acc[3], acc[7]))));
                 // P (bf16 pairs of this half's 64 keys) over the first 32 of its S columns: the A operand
                 // of O += P V reads keys 0-63 from the group's columns 0-31 and keys 64-127 from 64-95
                 ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));

@@ -360,6 +360,14 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// lo += the low bf16 of w, hi += its high bf16, each converted exactly (mixed-precision add): the row sums
+// of the softmax then add the very P values the PV product multiplies, not their fp32 originals.
+__device__ __forceinline__ void add_bf16x2(uint32_t w, float& lo, float& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tadd.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -16,6 +16,7 @@
 #include "score.cuh"
 #include "select.cuh"
 #include "attend.cuh"
+#include "attend_pair.cuh"
 #include "quant.cuh"
 
 namespace veda {
@@ -35,6 +36,7 @@ struct DeviceState {
     int sms = 0;
     int* err = nullptr;  // device address of g_err
     bool attend_attr[8] = {};  // (head_dim 128) + 2 * Q/K format; 6 + (head_dim 128) for the gather-free variant
+    bool pair_attr[4] = {};    // paired kernel: (head_dim 128) + 2 * gather-free
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -516,6 +518,104 @@ static int launch_attend(DeviceState* ds, const AttendMaps& maps, const AttendAr
     return launch_check("attend_kernel");
 }
 
+// Workspace of the paired attend: merged unit lists, their counts and the redo flags, each 256-aligned.
+struct PairWorkspace {
+    int32_t* units;
+    int2* counts;
+    int32_t* flags;
+};
+static int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+// sizes from the layout's video tile count, list width and tile count
+static int64_t pair_units_bytes(int64_t n_video, int64_t max_kept, int32_t n_heads) {
+    return align256(int64_t(n_heads) * ((n_video + 1) / 2) * 2 * max_kept * 4);
+}
+static int64_t pair_counts_bytes(int64_t n_video, int32_t n_heads) {
+    return align256(int64_t(n_heads) * ((n_video + 1) / 2) * 8);
+}
+static int64_t pair_flags_bytes(int64_t n_tiles, int32_t n_heads) { return align256(int64_t(n_heads) * n_tiles * 4); }
+static PairWorkspace pair_workspace(int64_t n_video, int64_t max_kept, int32_t n_heads, void* base) {
+    char* p = static_cast<char*>(base);
+    const int64_t ub = pair_units_bytes(n_video, max_kept, n_heads), cb = pair_counts_bytes(n_video, n_heads);
+    return {reinterpret_cast<int32_t*>(p), reinterpret_cast<int2*>(p + ub), reinterpret_cast<int32_t*>(p + ub + cb)};
+}
+
+extern "C" size_t veda_attend_paired_workspace_bytes(const veda_layout* layout, int32_t n_heads) {
+    if (!layout || n_heads <= 0) return 0;
+    const veda_layout_desc& d = layout->desc;
+    return size_t(pair_units_bytes(d.n_video, d.max_kept, n_heads) + pair_counts_bytes(d.n_video, n_heads) +
+                  pair_flags_bytes(d.n_tiles, n_heads));
+}
+
+// The paired attend: clear the redo flags, merge each pair's lists into units, run the paired kernel, then
+// the single-tile kernel over the query tiles it flagged (an empty pass when none is).
+template <int D, bool kDirect>
+static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, const int32_t* kept_idx,
+                         const int32_t* kept_cnt, void* workspace, cudaStream_t s) {
+    const PairWorkspace ws = pair_workspace(a.n_video, a.max_kept, a.n_heads, workspace);
+    cudaError_t e = cudaMemsetAsync(ws.flags, 0, size_t(a.n_heads) * size_t(a.n_tiles) * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(redo flags)");
+    PairUnitsArgs u{};
+    u.kept_idx = kept_idx;
+    u.kept_cnt = kept_cnt;
+    u.n_video = a.n_video;
+    u.max_kept = a.max_kept;
+    u.n_tiles = a.n_tiles;
+    u.n_heads = a.n_heads;
+    u.n_pairs = (a.n_video + 1) / 2;
+    u.units = ws.units;
+    u.counts = ws.counts;
+    u.err = a.err;
+    const int64_t warps = int64_t(u.n_heads) * u.n_pairs;
+    if (warps > 0) {
+        pair_units_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(u);
+        if (int rc = launch_check("pair_units_kernel")) return rc;
+    }
+    PairArgs p{};
+    p.units = ws.units;
+    p.counts = ws.counts;
+    p.ok_list = a.ok_list;
+    p.valid_count = a.valid_count;
+    p.perm = a.perm;
+    p.heads = a.heads;
+    p.out = a.out;
+    p.out_s0 = a.out_s0;
+    p.out_s1 = a.out_s1;
+    p.n_slots = a.n_slots;
+    p.max_kept = a.max_kept;
+    p.n_ok = a.n_ok;
+    p.n_tiles = a.n_tiles;
+    p.n_video = a.n_video;
+    p.n_global = a.n_global;
+    p.n_heads = a.n_heads;
+    p.h_total = a.h_total;
+    p.n_pairs = (a.n_video + 1) / 2;
+    p.n_gpairs = (a.n_global + 1) / 2;
+    p.n_items = a.n_heads * (p.n_pairs + p.n_gpairs);
+    p.scale_log2 = a.scale_log2;
+    p.timeout_ns = a.timeout_ns;
+    p.err = a.err;
+    p.hold_q = a.hold_q;
+    p.tile_coord = a.tile_coord;
+    p.tile_mask = a.tile_mask;
+    p.n_map_spans = a.n_map_spans;
+    p.q_row_sq = a.q_row_sq;
+    p.k_max_sq = a.k_max_sq;
+    p.seq_len = a.seq_len;
+    p.redo_flags = ws.flags;
+    using C = PairCfg<D>;
+    const int slot = (D == 128) + 2 * kDirect;
+    if (!ds->pair_attr[slot]) {
+        e = cudaFuncSetAttribute(attend_pair_kernel<D, kDirect>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_pair_kernel)");
+        ds->pair_attr[slot] = true;
+    }
+    attend_pair_kernel<D, kDirect><<<std::max(1, std::min(p.n_items, ds->sms)), C::kThreads, C::kSmem, s>>>(maps, p);
+    if (int rc = launch_check("attend_pair_kernel")) return rc;
+    a.redo_flags = ws.flags;
+    a.hold_q = 0;
+    return launch_attend<D, kQKBf16, kDirect>(ds, maps, a, s);
+}
+
 // The launch arguments both attend entry points share: lists, layout tables, output, limits and the wait
 // settings (tile tables and scales are left empty; each caller sets what its variant reads).
 static AttendArgs attend_args(const veda_layout_desc& d, const DeviceCopy* dc, const DeviceState* ds,
@@ -561,9 +661,9 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
                          const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
                          const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
                          const int32_t* heads, void* stream, int qk, const float* q_row_sq = nullptr,
-                         const float* k_max_sq = nullptr) {
+                         const float* k_max_sq = nullptr, void* pair_ws = nullptr) {
     const bool fp8 = qk != kQKBf16;  // 8-bit Q/K codes (e4m3 or int8)
-    const char* who = qk == kQKI8 ? "veda_attend_int8" : fp8 ? "veda_attend_fp8" : "veda_attend";
+    const char* who = qk == kQKI8 ? "veda_attend_int8" : fp8 ? "veda_attend_fp8" : pair_ws ? "veda_attend_paired" : "veda_attend";
     if (!layout || !q || !k || !v_t || !kept_idx || !kept_cnt || !out || !heads || (fp8 && (!sq || !sk)))
         return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
     if (fp8 ? dim != 128 : (dim != 64 && dim != 128))
@@ -593,6 +693,9 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
         a.k_max_sq = k_max_sq;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pair_ws)
+        return dim == 128 ? launch_paired<128, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s)
+                          : launch_paired<64, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
     if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, maps, a, s);
     if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, maps, a, s);
     return dim == 128 ? launch_attend<128, kQKBf16>(ds, maps, a, s) : launch_attend<64, kQKBf16>(ds, maps, a, s);
@@ -605,6 +708,30 @@ extern "C" int veda_attend(const veda_layout* layout, const void* q_t, const voi
     clear_error();
     return attend_common(layout, q_t, k_t, nullptr, nullptr, v_t, n_heads, dim, kept_idx, kept_cnt, out, out_strides,
                          h_total, heads, stream, kQKBf16, q_row_sq, k_max_sq);
+}
+
+// Checks shared by the paired entry points: the norms of the bound and an aligned workspace.
+static int check_paired(const char* who, const veda_layout* layout, int32_t n_heads, const float* q_row_sq,
+                        const float* k_max_sq, const void* workspace, size_t workspace_bytes) {
+    if (!q_row_sq || !k_max_sq)
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": the paired kernel needs q_row_sq and k_max_sq (veda_pool)");
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": workspace must be a 256-byte aligned device buffer");
+    if (layout && n_heads > 0 && workspace_bytes < veda_attend_paired_workspace_bytes(layout, n_heads))
+        return fail(VEDA_ERR_INVALID, std::string(who) + ": workspace smaller than veda_attend_paired_workspace_bytes");
+    return VEDA_OK;
+}
+
+extern "C" int veda_attend_paired(const veda_layout* layout, const void* q_t, const void* k_t, const void* v_t,
+                                  int32_t n_heads, int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt,
+                                  void* out, const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
+                                  const float* q_row_sq, const float* k_max_sq, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    clear_error();
+    if (int rc = check_paired("veda_attend_paired", layout, n_heads, q_row_sq, k_max_sq, workspace, workspace_bytes))
+        return rc;
+    return attend_common(layout, q_t, k_t, nullptr, nullptr, v_t, n_heads, dim, kept_idx, kept_cnt, out, out_strides,
+                         h_total, heads, stream, kQKBf16, q_row_sq, k_max_sq, workspace);
 }
 
 static_assert(kMapSets == kMaxDirectSpans + 1, "one map set per tiled span plus the global set");
@@ -645,14 +772,12 @@ static int make_row_map(CUtensorMap* m, const void* x, const int64_t st[3], int3
     return VEDA_OK;
 }
 
-extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
-                                  const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
-                                  int32_t h_total, int32_t dim, const int32_t* heads, int32_t n_heads,
-                                  const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
-                                  const int64_t out_strides[3], const float* q_row_sq, const float* k_max_sq,
-                                  void* stream) {
-    clear_error();
-    const char* who = "veda_attend_direct";
+static int attend_direct_impl(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
+                              const int64_t k_strides[3], const void* v, const int64_t v_strides[3], int32_t h_total,
+                              int32_t dim, const int32_t* heads, int32_t n_heads, const int32_t* kept_idx,
+                              const int32_t* kept_cnt, void* out, const int64_t out_strides[3], const float* q_row_sq,
+                              const float* k_max_sq, void* pair_ws, void* stream) {
+    const char* who = pair_ws ? "veda_attend_direct_paired" : "veda_attend_direct";
     if (!layout || !q || !k || !v || !kept_idx || !kept_cnt || !out || !heads)
         return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
     if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, std::string(who) + ": head_dim must be 64 or 128");
@@ -698,7 +823,36 @@ extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, cons
         a.k_max_sq = k_max_sq;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pair_ws)
+        return dim == 128 ? launch_paired<128, true>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s)
+                          : launch_paired<64, true>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
     return dim == 128 ? launch_attend<128, kQKBf16, true>(ds, maps, a, s) : launch_attend<64, kQKBf16, true>(ds, maps, a, s);
+}
+
+extern "C" int veda_attend_direct(const veda_layout* layout, const void* q, const int64_t q_strides[3], const void* k,
+                                  const int64_t k_strides[3], const void* v, const int64_t v_strides[3],
+                                  int32_t h_total, int32_t dim, const int32_t* heads, int32_t n_heads,
+                                  const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                                  const int64_t out_strides[3], const float* q_row_sq, const float* k_max_sq,
+                                  void* stream) {
+    clear_error();
+    return attend_direct_impl(layout, q, q_strides, k, k_strides, v, v_strides, h_total, dim, heads, n_heads, kept_idx,
+                              kept_cnt, out, out_strides, q_row_sq, k_max_sq, nullptr, stream);
+}
+
+extern "C" int veda_attend_direct_paired(const veda_layout* layout, const void* q, const int64_t q_strides[3],
+                                         const void* k, const int64_t k_strides[3], const void* v,
+                                         const int64_t v_strides[3], int32_t h_total, int32_t dim,
+                                         const int32_t* heads, int32_t n_heads, const int32_t* kept_idx,
+                                         const int32_t* kept_cnt, void* out, const int64_t out_strides[3],
+                                         const float* q_row_sq, const float* k_max_sq, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+    clear_error();
+    if (int rc = check_paired("veda_attend_direct_paired", layout, n_heads, q_row_sq, k_max_sq, workspace,
+                              workspace_bytes))
+        return rc;
+    return attend_direct_impl(layout, q, q_strides, k, k_strides, v, v_strides, h_total, dim, heads, n_heads, kept_idx,
+                              kept_cnt, out, out_strides, q_row_sq, k_max_sq, workspace, stream);
 }
 
 extern "C" int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* k_codes,

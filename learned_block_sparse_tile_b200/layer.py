@@ -29,13 +29,18 @@ class VedaLayer:
     logit_bound  bf16 paths: the pool/gather of Q also writes ||q||^2 per row and that of K the largest
                  ||k||^2 per head, and the attend takes them as its logit bound (later tiles of an item may
                  then skip the row max; same softmax). Default True; the 8-bit paths ignore it
+    paired       with the logit bound: the paired attend (veda_attend_paired / veda_attend_direct_paired),
+                 two neighbouring query tiles per work item sharing each kept K/V tile load, the softmax
+                 reference fixed by the bound, and an exact redo of any query tile the bound cannot serve.
+                 Default True; False keeps the single-tile attend
     """
 
     LAUNCHES_PER_GROUP = 7  # tile-order path: gather q, gather k, 2 score GEMMs, select, gather v, attend
     LAUNCHES_PER_GROUP_DIRECT = 6  # gather-free path: pool q, pool k, 2 score GEMMs, select, attend
+    EXTRA_LAUNCHES_PAIRED = 2  # the paired attend adds the list merge and the (usually empty) redo pass
 
     def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False,
-                 int8_qk=False, direct=None, logit_bound=True):
+                 int8_qk=False, direct=None, logit_bound=True, paired=True):
         self.seq_len, self.heads, self.dim = int(seq_len), int(heads), int(dim)
         if fp8_qk and int8_qk:
             raise ValueError("VedaLayer: choose one of fp8_qk and int8_qk")
@@ -58,6 +63,7 @@ class VedaLayer:
                     L.veda_layout_export_direct(x)  # raises with the reason
         self.direct = bool(direct)
         self.logit_bound = bool(logit_bound) and not (self.fp8_qk or self.int8_qk)
+        self.paired = bool(paired) and self.logit_bound
         self.groups = []
         for box in sorted(groups):
             lay = layouts[box]
@@ -89,8 +95,10 @@ class VedaLayer:
                          k_max_sq=torch.empty(n, dtype=torch.float32, device=dev))
             else:
                 g.update(q_row_sq=None, k_max_sq=None)
+            g.update(pair_ws=L.paired_workspace(lay, n, dev) if self.paired else None)
             self.groups.append(g)
-        self.launches = (self.LAUNCHES_PER_GROUP_DIRECT if self.direct else self.LAUNCHES_PER_GROUP) * len(self.groups)
+        self.launches = ((self.LAUNCHES_PER_GROUP_DIRECT if self.direct else self.LAUNCHES_PER_GROUP) +
+                         (self.EXTRA_LAUNCHES_PAIRED if self.paired else 0)) * len(self.groups)
         self._side = torch.cuda.Stream(self.device)  # the V gathers
 
     def set_projections(self, proj_q, proj_k):
@@ -164,8 +172,12 @@ class VedaLayer:
                 L.veda_select(lay, g["scores"], g["kept_idx"], g["kept_cnt"], st)
                 done(m, st)
                 m = mark("attend", st)
-                L.veda_attend_direct(lay, q, k, v, g["kept_idx"], g["kept_cnt"], out, g["heads"], st,
-                                     q_row_sq=g["q_row_sq"], k_max_sq=g["k_max_sq"])
+                if self.paired:
+                    L.veda_attend_direct_paired(lay, q, k, v, g["kept_idx"], g["kept_cnt"], out, g["heads"],
+                                                g["q_row_sq"], g["k_max_sq"], g["pair_ws"], st)
+                else:
+                    L.veda_attend_direct(lay, q, k, v, g["kept_idx"], g["kept_cnt"], out, g["heads"], st,
+                                         q_row_sq=g["q_row_sq"], k_max_sq=g["k_max_sq"])
                 done(m, st)
                 continue
             m = mark("gather_qk", st)
@@ -196,6 +208,9 @@ class VedaLayer:
             if self.fp8_qk or self.int8_qk:
                 attend = L.veda_attend_int8 if self.int8_qk else L.veda_attend_fp8
                 attend(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
+            elif self.paired:
+                L.veda_attend_paired(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"],
+                                     g["q_row_sq"], g["k_max_sq"], g["pair_ws"], st)
             else:
                 L.veda_attend(lay, g["q_t"], g["k_t"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st,
                               q_row_sq=g["q_row_sq"], k_max_sq=g["k_max_sq"])

@@ -39,17 +39,20 @@ def built():
     _inputs.clear()
 
 
-# the layer's own path choice (gather-free wherever the layout has a box form, as bench.py runs it), and
-# the tile-order path on two of the configurations
-@pytest.mark.parametrize("name,direct", [(n, None) for n in ["single", "mixed", "long", "sweep_tiles24", "sweep_r025",
-                                                             "sweep_r050", "sweep_dense", "sweep_fp8", "sweep_int8"]]
-                         + [("single", False), ("mixed", False)])
-def test_full_size_layer(name, direct):
+# the layer's own path choice (gather-free wherever the layout has a box form, and the paired attend with
+# the logit bound, as bench.py runs it), the tile-order path on two of the configurations, and the
+# single-tile attend on the 104k layer
+@pytest.mark.parametrize("name,direct,paired",
+                         [(n, None, True) for n in ["single", "mixed", "long", "sweep_tiles24", "sweep_r025",
+                                                    "sweep_r050", "sweep_dense", "sweep_fp8", "sweep_int8"]]
+                         + [("single", False, True), ("mixed", False, True), ("single", None, False)])
+def test_full_size_layer(name, direct, paired):
     wl = V.workload(name)
     x = inputs(wl)
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk, direct=direct)
+                      wl.heads, wl.dim, fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk, direct=direct, paired=paired)
     assert layer.direct == (direct is None and not (wl.fp8_qk or wl.int8_qk))
+    assert layer.paired == (paired and not (wl.fp8_qk or wl.int8_qk))
     layer.set_projections(x["pq"], x["pk"])
     out = torch.full_like(x["dq"], 7.0)
     layer.forward(x["dq"], x["dk"], x["dv"], out)
@@ -174,13 +177,19 @@ def _sampled_error(got, want_t, lay_o, heads, q_tiles, packed=True):
 
 def test_full_size_paths_agree_bit_for_bit():
     # on the 104k layer every tile is a full box, so the gather-free attend sees the keys in the same order
-    # as the tile-order one: the two paths give the same features, lists and output, bit for bit
+    # as the tile-order one: the two paths give the same features, lists and output, bit for bit (with the
+    # paired attend, the layer's default, and with the single-tile one)
     wl = V.workload("single")
     x = inputs(wl)
+    for paired in (True, False):
+        _paths_agree(wl, x, paired)
+
+
+def _paths_agree(wl, x, paired):
     outs = []
     for direct in (True, False):
         layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
-                          wl.heads, wl.dim, direct=direct)
+                          wl.heads, wl.dim, direct=direct, paired=paired)
         layer.set_projections(x["pq"], x["pk"])
         out = torch.full_like(x["dq"], 7.0)
         layer.forward(x["dq"], x["dk"], x["dv"], out)

@@ -92,9 +92,10 @@ struct AttendArgs {
     const float* q_row_sq;  // [n_heads, seq_len]
     const float* k_max_sq;  // [n_heads]
     int64_t seq_len;
-    // redo pass after the paired kernel (attend_pair.cuh): when set, only the query tiles (head index, tile)
-    // flagged non-zero in [n_heads, n_tiles] are processed; every other item is skipped by every role
-    const int32_t* redo_flags;
+    // redo pass after the paired kernel (attend_pair.cuh): when set, the kernel processes only the items
+    // redo_items[0, *redo_count) (device memory, written by the kernel before it) instead of all n_items
+    const int32_t* redo_items;
+    const int32_t* redo_count;
 };
 
 // With the logit bound, a softmax group takes its reference m from the exact row maxima of its first tile
@@ -197,9 +198,12 @@ __device__ __forceinline__ int item_tiles(const AttendArgs& a, int hh, int qt, c
     return n;
 }
 
-// True when a redo pass skips this query tile (see AttendArgs::redo_flags). Uniform across the CTA.
-__device__ __forceinline__ bool item_skipped(const AttendArgs& a, int hh, int qt) {
-    return a.redo_flags != nullptr && __ldg(a.redo_flags + int64_t(hh) * a.n_tiles + qt) == 0;
+// Items of this launch: all n_items, or the redo list's length. Item i is then i, or redo_items[i].
+__device__ __forceinline__ int launch_items(const AttendArgs& a) {
+    return a.redo_count != nullptr ? *a.redo_count : a.n_items;
+}
+__device__ __forceinline__ int item_at(const AttendArgs& a, int i) {
+    return a.redo_items != nullptr ? a.redo_items[i] : i;
 }
 
 // Item order: the dense global query tiles first (they are the longest), then head-major video tiles,
@@ -234,6 +238,8 @@ __global__ void __launch_bounds__(640, 1)
     constexpr int KS = C::kKStages, VS = C::kVStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw;
+    const int n_items = launch_items(a);
+    if (int(blockIdx.x) >= n_items) return;  // uniform: a redo pass with fewer items than CTAs
     if ((ptx::smem_addr(smem) & 1023) != 0) {  // the swizzled tiles need a 1024-byte aligned base
         if (threadIdx.x == 0) atomicOr(a.err, kErrLayout);
         return;
@@ -298,10 +304,9 @@ __global__ void __launch_bounds__(640, 1)
         const int S = kq ? KS : VS;
         const uint64_t keep = ptx::policy_evict_last();
         int issued_q = 0, issued = 0;  // copies issued so far (warp-uniform): Q tiles; K or V tiles
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+        for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
             int hh, qt;
-            decode_item(a, item, &hh, &qt);
-            if (item_skipped(a, hh, qt)) continue;
+            decode_item(a, item_at(a, i), &hh, &qt);
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
@@ -401,10 +406,9 @@ __global__ void __launch_bounds__(640, 1)
         const uint64_t dq = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffQ), 16, 1024);
         const uint64_t dk = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffK), 16, 1024);
         const uint64_t dv = ptx::smem_desc_sw128(ptx::smem_addr(smem + C::kOffV), 16384, 1024);
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+        for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
             int hh, qt;
-            decode_item(a, item, &hh, &qt);
-            if (item_skipped(a, hh, qt)) continue;
+            decode_item(a, item_at(a, i), &hh, &qt);
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);
@@ -513,10 +517,9 @@ __global__ void __launch_bounds__(640, 1)
         int od_mine = 0, od_other = 0;  // o_done phases of this group and the other: one per item with a tile
         const bool releaser = (sw & 7) == 0 && lane == 0;  // one thread per group frees K slots
         constexpr int kCols = D / 4;  // output columns each thread writes (four threads per row)
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+        for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
             int hh, qt;
-            decode_item(a, item, &hh, &qt);
-            if (item_skipped(a, hh, qt)) continue;
+            decode_item(a, item_at(a, i), &hh, &qt);
             const int32_t* list;
             bool bad;
             const int n = item_tiles(a, hh, qt, &list, &bad);

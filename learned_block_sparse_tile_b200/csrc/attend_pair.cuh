@@ -15,8 +15,8 @@
 // taken and O is never rescaled. That lets both softmax groups add into one O per query tile (the
 // single-tile kernel keeps one O per group and merges them). The result is the same softmax; only when
 // the bound is loose by more than kBoundOffset + 60 (log2 units) would the row's largest P drop below
-// 2^-60 - the row sum tells - and the query tile is then flagged for a redo by the single-tile kernel's
-// exact path (attend_kernel with AttendArgs::redo_flags), which rewrites all of its rows.
+// 2^-60 - the row sum tells - and the query tile is then listed for a redo by the single-tile kernel's
+// exact path (attend_kernel over AttendArgs::redo_items), which rewrites all of its rows.
 //
 // Roles (640 threads, one persistent CTA per SM, one pair item at a time):
 //   warp 0       TMA producer of the two Q tiles (one buffer pair) and the union's K tiles (ring);
@@ -58,8 +58,9 @@ struct PairUnitsArgs {
 };
 
 // Length of the valid prefix of a kept list: count within [0, max_kept], ids in [0, n_tiles), strictly
-// ascending; *bad when anything was cut. Warp-collective.
-__device__ __forceinline__ int checked_list_len(const int32_t* l, int cnt, int max_kept, int n_tiles, bool* bad) {
+// ascending; *bad when anything was cut. The valid entries are copied to dst. Warp-collective.
+__device__ __forceinline__ int load_checked_list(const int32_t* l, int cnt, int max_kept, int n_tiles, bool* bad,
+                                                 int32_t* dst) {
     const int lane = threadIdx.x & 31;
     bool b = false;
     if (cnt < 0 || cnt > max_kept) {
@@ -76,9 +77,11 @@ __device__ __forceinline__ int checked_list_len(const int32_t* l, int cnt, int m
         const unsigned badmask = __ballot_sync(0xffffffffu, !ok);
         if (badmask) {
             n = base + __ffs(badmask) - 1;
+            if (j < n) dst[j] = v;
             b = true;
             break;
         }
+        if (j < cnt) dst[j] = v;
         prev_last = __shfl_sync(0xffffffffu, v, 31);
     }
     *bad = b;
@@ -90,7 +93,7 @@ __device__ __forceinline__ int count_below(const int32_t* l, int n, int v) {
     int lo = 0, hi = n;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (__ldg(l + mid) < v)
+        if (l[mid] < v)
             lo = mid + 1;
         else
             hi = mid;
@@ -98,33 +101,39 @@ __device__ __forceinline__ int count_below(const int32_t* l, int n, int v) {
     return lo;
 }
 
-// One warp per (head, pair of video query tiles 2p, 2p + 1): the checked lists of both rows merged into
-// units. Unit (t, A) lands at (entries of A below t) + (entries of B below t), unit (t, B) at (entries of
-// A up to t) + (entries of B below t), so a tile in both lists gives (t, A), (t, B) next to each other.
+// One warp per (head, pair of video query tiles 2p, 2p + 1): the checked lists of both rows, staged in
+// the warp's slice of shared memory (2 max_kept entries), merged into units. Unit (t, A) lands at
+// (entries of A below t) + (entries of B below t), unit (t, B) at (entries of A up to t) + (entries of B
+// below t), so a tile in both lists gives (t, A), (t, B) next to each other.
 __global__ void __launch_bounds__(256) pair_units_kernel(const PairUnitsArgs a) {
+    extern __shared__ int32_t staged[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t gw = int64_t(blockIdx.x) * 8 + warp;
-    if (gw >= int64_t(a.n_heads) * a.n_pairs) return;
+    const int64_t gw = int64_t(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (gw >= int64_t(a.n_heads) * a.n_pairs) return;  // whole warps
     const int hh = int(gw / a.n_pairs), p = int(gw % a.n_pairs);
     const int64_t row_a = int64_t(hh) * a.n_video + 2 * p;
     const bool has_b = 2 * p + 1 < a.n_video;
+    int32_t* sa = staged + int64_t(warp) * 2 * a.max_kept;
+    int32_t* sb = sa + a.max_kept;
     const int32_t* la = a.kept_idx + row_a * a.max_kept;
-    const int32_t* lb = la + a.max_kept;
     bool bad_a = false, bad_b = false;
-    const int na = checked_list_len(la, __ldg(a.kept_cnt + row_a), a.max_kept, a.n_tiles, &bad_a);
-    const int nb = has_b ? checked_list_len(lb, __ldg(a.kept_cnt + row_a + 1), a.max_kept, a.n_tiles, &bad_b) : 0;
+    const int na = load_checked_list(la, __ldg(a.kept_cnt + row_a), a.max_kept, a.n_tiles, &bad_a, sa);
+    const int nb = has_b ? load_checked_list(la + a.max_kept, __ldg(a.kept_cnt + row_a + 1), a.max_kept, a.n_tiles,
+                                             &bad_b, sb)
+                         : 0;
     if ((bad_a || bad_b) && lane == 0) atomicOr(a.err, kErrBadList);
+    __syncwarp();
     int32_t* out = a.units + gw * (2 * int64_t(a.max_kept));
     for (int i = lane; i < na; i += 32) {
-        const int t = __ldg(la + i);
-        const int below = count_below(lb, nb, t);
-        const bool both = below < nb && __ldg(lb + below) == t;
+        const int t = sa[i];
+        const int below = count_below(sb, nb, t);
+        const bool both = below < nb && sb[below] == t;
         out[i + below] = (t << 3) | (both ? 0 : 4) | 2;
     }
     for (int j = lane; j < nb; j += 32) {
-        const int t = __ldg(lb + j);
-        const int upto = count_below(la, na, t + 1);
-        const bool both = upto > 0 && __ldg(la + upto - 1) == t;
+        const int t = sb[j];
+        const int upto = count_below(sa, na, t + 1);
+        const bool both = upto > 0 && sa[upto - 1] == t;
         out[upto + j] = (t << 3) | 4 | (both ? 0 : 2) | 1;
     }
     if (lane == 0) a.counts[gw] = make_int2(na + nb, na);
@@ -154,7 +163,11 @@ struct PairArgs {
     const float* q_row_sq;  // [n_heads, seq_len]
     const float* k_max_sq;  // [n_heads]
     int64_t seq_len;
-    int32_t* redo_flags;  // [n_heads, n_tiles], zero on entry; set for query tiles that need the exact redo
+    // query tiles that need the exact redo: a flag per (head index, tile) (zero on entry) and the list of
+    // their single-tile item numbers (attend.cuh's order) with its length (zero on entry)
+    int32_t* redo_flags;  // [n_heads, n_tiles]
+    int32_t* redo_items;  // [n_heads * n_tiles]
+    int32_t* redo_count;
 };
 
 struct PairItem {
@@ -612,8 +625,13 @@ __global__ void __launch_bounds__(640, 1)
             const bool have = n_out > 0;
             // a real row whose sum left [2^-60, 2^100] (or is NaN): the exact redo rewrites its query tile
             const bool redo = prow >= 0 && have && !(l >= kRedoBelow && l <= kRedoAbove);
-            if (__any_sync(0xffffffffu, redo) && lane == 0)
-                atomicOr(a.redo_flags + int64_t(pi.hh) * a.n_tiles + qt_out, 1);
+            if (__any_sync(0xffffffffu, redo) && lane == 0 &&
+                atomicOr(a.redo_flags + int64_t(pi.hh) * a.n_tiles + qt_out, 1) == 0) {
+                // the first warp to flag the tile lists it
+                const int single = qt_out >= a.n_video ? pi.hh * a.n_global + (qt_out - a.n_video)
+                                                       : a.n_heads * a.n_global + pi.hh * a.n_video + qt_out;
+                a.redo_items[atomicAdd(a.redo_count, 1)] = single;
+            }
             const float inv = l > 0.f ? 1.f / l : 0.f;
             ptx::tc_fence_after();
             // this thread's half of the row is read (and scaled into bf16 pairs) before O is released to the

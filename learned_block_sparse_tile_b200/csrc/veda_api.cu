@@ -518,11 +518,14 @@ static int launch_attend(DeviceState* ds, const AttendMaps& maps, const AttendAr
     return launch_check("attend_kernel");
 }
 
-// Workspace of the paired attend: merged unit lists, their counts and the redo flags, each 256-aligned.
+// Workspace of the paired attend, each region 256-aligned: the merged unit lists and their counts, the
+// redo flags followed by the redo list's length (cleared together), and the redo list.
 struct PairWorkspace {
     int32_t* units;
     int2* counts;
     int32_t* flags;
+    int32_t* redo_count;
+    int32_t* redo_items;
 };
 static int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 // sizes from the layout's video tile count, list width and tile count
@@ -533,17 +536,22 @@ static int64_t pair_counts_bytes(int64_t n_video, int32_t n_heads) {
     return align256(int64_t(n_heads) * ((n_video + 1) / 2) * 8);
 }
 static int64_t pair_flags_bytes(int64_t n_tiles, int32_t n_heads) { return align256(int64_t(n_heads) * n_tiles * 4); }
-static PairWorkspace pair_workspace(int64_t n_video, int64_t max_kept, int32_t n_heads, void* base) {
+static int64_t pair_workspace_total(int64_t n_video, int64_t max_kept, int64_t n_tiles, int32_t n_heads) {
+    return pair_units_bytes(n_video, max_kept, n_heads) + pair_counts_bytes(n_video, n_heads) +
+           2 * pair_flags_bytes(n_tiles, n_heads) + 256;
+}
+static PairWorkspace pair_workspace(int64_t n_video, int64_t max_kept, int64_t n_tiles, int32_t n_heads, void* base) {
     char* p = static_cast<char*>(base);
     const int64_t ub = pair_units_bytes(n_video, max_kept, n_heads), cb = pair_counts_bytes(n_video, n_heads);
-    return {reinterpret_cast<int32_t*>(p), reinterpret_cast<int2*>(p + ub), reinterpret_cast<int32_t*>(p + ub + cb)};
+    const int64_t fb = pair_flags_bytes(n_tiles, n_heads);
+    return {reinterpret_cast<int32_t*>(p), reinterpret_cast<int2*>(p + ub), reinterpret_cast<int32_t*>(p + ub + cb),
+            reinterpret_cast<int32_t*>(p + ub + cb + fb), reinterpret_cast<int32_t*>(p + ub + cb + fb + 256)};
 }
 
 extern "C" size_t veda_attend_paired_workspace_bytes(const veda_layout* layout, int32_t n_heads) {
     if (!layout || n_heads <= 0) return 0;
     const veda_layout_desc& d = layout->desc;
-    return size_t(pair_units_bytes(d.n_video, d.max_kept, n_heads) + pair_counts_bytes(d.n_video, n_heads) +
-                  pair_flags_bytes(d.n_tiles, n_heads));
+    return size_t(pair_workspace_total(d.n_video, d.max_kept, d.n_tiles, n_heads));
 }
 
 // The paired attend: clear the redo flags, merge each pair's lists into units, run the paired kernel, then
@@ -551,8 +559,8 @@ extern "C" size_t veda_attend_paired_workspace_bytes(const veda_layout* layout, 
 template <int D, bool kDirect>
 static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, const int32_t* kept_idx,
                          const int32_t* kept_cnt, void* workspace, cudaStream_t s) {
-    const PairWorkspace ws = pair_workspace(a.n_video, a.max_kept, a.n_heads, workspace);
-    cudaError_t e = cudaMemsetAsync(ws.flags, 0, size_t(a.n_heads) * size_t(a.n_tiles) * 4, s);
+    const PairWorkspace ws = pair_workspace(a.n_video, a.max_kept, a.n_tiles, a.n_heads, workspace);
+    cudaError_t e = cudaMemsetAsync(ws.flags, 0, size_t(pair_flags_bytes(a.n_tiles, a.n_heads)) + 256, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(redo flags)");
     PairUnitsArgs u{};
     u.kept_idx = kept_idx;
@@ -567,7 +575,18 @@ static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, 
     u.err = a.err;
     const int64_t warps = int64_t(u.n_heads) * u.n_pairs;
     if (warps > 0) {
-        pair_units_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(u);
+        // each warp stages its two lists in shared memory: up to 8 warps per block within 48 KB, else one
+        // warp per block with the opt-in size (lists of up to ~29,000 tiles)
+        const int64_t per_warp = 8 * int64_t(std::max(u.max_kept, 1));
+        const int wpb = int(std::max<int64_t>(1, std::min<int64_t>(8, 49152 / per_warp)));
+        const int64_t smem = per_warp * wpb;
+        if (smem > 227 * 1024)
+            return fail(VEDA_ERR_UNSUPPORTED, "veda_attend_paired: kept lists too wide for the list merge");
+        if (smem > 49152) {
+            e = cudaFuncSetAttribute(pair_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(pair_units_kernel)");
+        }
+        pair_units_kernel<<<unsigned((warps + wpb - 1) / wpb), unsigned(32 * wpb), size_t(smem), s>>>(u);
         if (int rc = launch_check("pair_units_kernel")) return rc;
     }
     PairArgs p{};
@@ -602,6 +621,8 @@ static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, 
     p.k_max_sq = a.k_max_sq;
     p.seq_len = a.seq_len;
     p.redo_flags = ws.flags;
+    p.redo_items = ws.redo_items;
+    p.redo_count = ws.redo_count;
     using C = PairCfg<D>;
     const int slot = (D == 128) + 2 * kDirect;
     if (!ds->pair_attr[slot]) {
@@ -611,7 +632,9 @@ static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, 
     }
     attend_pair_kernel<D, kDirect><<<std::max(1, std::min(p.n_items, ds->sms)), C::kThreads, C::kSmem, s>>>(maps, p);
     if (int rc = launch_check("attend_pair_kernel")) return rc;
-    a.redo_flags = ws.flags;
+    // the redo pass over the listed items (at most n_items); CTAs past the list's length return at once
+    a.redo_items = ws.redo_items;
+    a.redo_count = ws.redo_count;
     a.hold_q = 0;
     return launch_attend<D, kQKBf16, kDirect>(ds, maps, a, s);
 }

@@ -56,11 +56,23 @@ def oracle_out(c, box, heads, res, q, k, v, want, idx=None, cnt=None):
 
 def redo_flags(lay, n, ws):
     """The redo flags the paired launch left in its workspace ([n, n_tiles] int32 after the merged lists and
-    their counts, each region 256-byte aligned)."""
+    their counts, each region 256-byte aligned), checked against the redo list that follows them: its
+    length (an int32 in a 256-byte slot) and its entries (single-tile item numbers: global query tiles
+    first, head-major, then video ones)."""
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
     pairs = (lay.n_video + 1) // 2
     off = a256(n * pairs * 2 * lay.max_kept * 4) + a256(n * pairs * 8)
-    return ws[off:off + n * lay.n_tiles * 4].view(torch.int32).view(n, lay.n_tiles).cpu().numpy()
+    fb = a256(n * lay.n_tiles * 4)
+    flags = ws[off:off + n * lay.n_tiles * 4].view(torch.int32).view(n, lay.n_tiles).cpu().numpy()
+    count = int(ws[off + fb:off + fb + 4].view(torch.int32).item())
+    items = ws[off + fb + 256:off + fb + 256 + 4 * count].view(torch.int32).cpu().numpy()
+    want = []
+    for hh in range(n):
+        for t in np.flatnonzero(flags[hh]):
+            want.append(hh * lay.n_global + (t - lay.n_video) if t >= lay.n_video
+                        else n * lay.n_global + hh * lay.n_video + t)
+    assert sorted(items.tolist()) == sorted(want), (items, want)
+    return flags
 
 
 @pytest.mark.parametrize("name", SMALL)

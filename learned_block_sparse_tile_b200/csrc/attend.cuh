@@ -637,7 +637,6 @@ __global__ void __launch_bounds__(640, 1)
                 const float negm = m_ref == -INFINITY ? 0.f : -m_ref;
                 const uint64_t negm2 = ptx::f2_pack(negm, negm);
                 // row sums over the bf16 P the PV product reads (eight independent chains)
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
                     const uint64_t x = ptx::f2_fma(ptx::f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2x2, negm2);
@@ -651,33 +650,40 @@ __global__ void __launch_bounds__(640, 1)
                         p1 = ptx::ex2(x1);
                     }
                     s[c >> 1] = ptx::pack_bf16(p0, p1);
-                    ptx::add_bf16x2(s[c >> 1], acc[(c >> 1) & 3], acc[4 + ((c >> 1) & 3)]);
                 }
-                lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(ptx::f2_pack(acc[0], acc[4]), ptx::f2_pack(acc[1], acc[5])),
-                                                     ptx::f2_add(ptx::f2_pack(acc[2], acc[6]), ptx::f2_pack(acc[3], acc[7]))));
+                // the row sum over the bf16 P the PV product reads (eight independent chains); lsum was scaled
+                // with O above when the reference moved
+                auto add_row_sum = [&]() {
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) ptx::add_bf16x2(s[c], acc[c & 3], acc[4 + (c & 3)]);
+                    lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(ptx::f2_pack(acc[0], acc[4]), ptx::f2_pack(acc[1], acc[5])),
+                                                         ptx::f2_add(ptx::f2_pack(acc[2], acc[6]), ptx::f2_pack(acc[3], acc[7]))));
+                };
                 // P (bf16 pairs of this half's 64 keys) over the first 32 of its S columns: the A operand
                 // of O += P V reads keys 0-63 from the group's columns 0-31 and keys 64-127 from 64-95
                 ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
                 ptx::tmem_wait_st();
-                if (k > 0) {
+                const bool rescale = k > 0 && __any_sync(0xffffffffu, resc);
+                if (rescale) {
                     // a new reference: rescale this half's share of the accumulator's columns before P is
-                    // handed over (P is stored first, so its registers are free here)
-                    if (__any_sync(0xffffffffu, resc)) {
+                    // handed over (the row sum is taken first, so P's registers are free here)
+                    add_row_sum();
 #pragma unroll 1
-                        for (int i = 0; i < D / 64; ++i) {
-                            uint32_t o[32];
-                            const uint32_t ta = t_o + (D / 2) * half + 32 * i;
-                            ptx::tmem_ld32(ta, o);
-                            ptx::tmem_wait_ld();
+                    for (int i = 0; i < D / 64; ++i) {
+                        uint32_t o[32];
+                        const uint32_t ta = t_o + (D / 2) * half + 32 * i;
+                        ptx::tmem_ld32(ta, o);
+                        ptx::tmem_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                            ptx::tmem_st32(ta, o);
-                        }
-                        ptx::tmem_wait_st();
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        ptx::tmem_st32(ta, o);
                     }
+                    ptx::tmem_wait_st();
                 }
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&B.p_full[w]);
+                if (!rescale) add_row_sum();  // off the path to the PV
             }
             if (!ok) break;
             // both groups' last PVs of this item must be complete before either accumulator is read. This

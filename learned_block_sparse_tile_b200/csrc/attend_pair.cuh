@@ -576,8 +576,6 @@ __global__ void __launch_bounds__(640, 1)
                 }
                 const float negm = (u & 1) ? negm_b : negm_a;
                 const uint64_t negm2 = ptx::f2_pack(negm, negm);
-                // row sums over the bf16 P the PV product reads (eight independent chains)
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
                     const uint64_t x =
@@ -592,18 +590,22 @@ __global__ void __launch_bounds__(640, 1)
                         p1 = ptx::ex2(x1);
                     }
                     s[c >> 1] = ptx::pack_bf16(p0, p1);
-                    ptx::add_bf16x2(s[c >> 1], acc[(c >> 1) & 3], acc[4 + ((c >> 1) & 3)]);
                 }
+                ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&B.p_full[w]);
+                // the row sums come after the hand-off, off the path to the PV: over the bf16 P the PV
+                // product reads (eight independent chains)
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 32; ++c) ptx::add_bf16x2(s[c], acc[c & 3], acc[4 + (c & 3)]);
                 const uint64_t tot = ptx::f2_add(ptx::f2_add(ptx::f2_pack(acc[0], acc[4]), ptx::f2_pack(acc[1], acc[5])),
                                                  ptx::f2_add(ptx::f2_pack(acc[2], acc[6]), ptx::f2_pack(acc[3], acc[7])));
                 if (u & 1)
                     sum_b = ptx::f2_add(sum_b, tot);
                 else
                     sum_a = ptx::f2_add(sum_a, tot);
-                ptx::tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(&B.p_full[w]);
             }
             if (!ok) break;
             ok = ptx::mbar_wait(&B.o_done, it & 1, abort_flag, tmo);  // every PV of the item is complete

@@ -401,6 +401,12 @@ void veda_set_wait_timeout_ns(uint64_t ns);
  * VEDA_ERR_TIMEOUT. The output of that call is unspecified; the device stays usable. */
 void veda_debug_hold_next_attend(void);
 
+/* Test hook (the pages have no counterpart): caps the number of CTAs of the calling thread's attend
+ * launches (every variant, and both kernels of the paired ones) at n, so that each CTA of a small case
+ * walks many work items in a row, as on a full-size layer; n <= 0 removes the cap. Results do not
+ * depend on it. */
+void veda_debug_attend_ctas(int32_t n);
+
 /* Test hook for the attend kernel's exponentials (the pages have no counterpart): evaluates, for each of
  * n fp32 inputs x, the three forms of 2^x the library has on the device: the FMA-pipe polynomial the
  * attend softmax uses for part of its columns (Cody-Waite reduction plus a cubic; inputs below -126 are

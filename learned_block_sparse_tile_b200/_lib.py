@@ -24,7 +24,7 @@ EXPORTS = [
     "veda_debug_hold_next_attend", "veda_quantize_fp8", "veda_gather_fp8", "veda_attend_fp8",
     "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8", "veda_layout_export_direct", "veda_pool",
     "veda_attend_direct", "veda_debug_exp2", "veda_grid_of", "veda_describe_packed_layout",
-    "veda_attend_paired_workspace_bytes", "veda_attend_paired", "veda_attend_direct_paired",
+    "veda_attend_paired_workspace_bytes", "veda_attend_paired", "veda_attend_direct_paired", "veda_debug_attend_ctas",
 ]
 
 VEDA_SEG_OTHER, VEDA_SEG_VIDEO, VEDA_SEG_COND, VEDA_SEG_REF_IMG = range(4)
@@ -122,6 +122,8 @@ def lib():
         L.veda_debug_hold_next_attend.argtypes = []
         L.veda_debug_hold_next_attend.restype = None
         L.veda_debug_exp2.argtypes = [p, p, p, p, i64, vp]
+        L.veda_debug_attend_ctas.argtypes = [i32]
+        L.veda_debug_attend_ctas.restype = None
         L.veda_grid_of.argtypes = [p, i64, i64, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
         L.veda_describe_packed_layout.argtypes = [C.POINTER(Segment), i32, i64, C.POINTER(C.c_int32), p,
                                                   C.POINTER(PackedDesc)]
@@ -370,6 +372,11 @@ def veda_set_wait_timeout_ns(ns):
 def veda_debug_hold_next_attend():
     """Test hook: the calling thread's next veda_attend withholds its Q loads (its waits expire)."""
     lib().veda_debug_hold_next_attend()
+
+
+def veda_debug_attend_ctas(n):
+    """Test hook: caps the CTAs of this thread's attend launches at n (0 removes the cap)."""
+    lib().veda_debug_attend_ctas(int(n))
 
 
 def veda_debug_exp2(x, poly=None, mufu=None, exp2f_out=None, stream=None):

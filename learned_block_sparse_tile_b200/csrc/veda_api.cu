@@ -29,6 +29,7 @@ namespace {
 
 thread_local std::string t_error;
 thread_local bool t_hold_next_attend = false;
+thread_local int t_attend_ctas = 0;  // test hook: cap on the CTAs of this thread's attend launches (0: none)
 std::atomic<uint64_t> g_timeout_ns{1000000000ull};
 
 struct DeviceState {
@@ -160,6 +161,13 @@ extern "C" const char* veda_last_error(void) { return t_error.c_str(); }
 extern "C" void veda_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : 1; }
 
 extern "C" void veda_debug_hold_next_attend(void) { t_hold_next_attend = true; }
+extern "C" void veda_debug_attend_ctas(int32_t n) { t_attend_ctas = n > 0 ? n : 0; }
+
+// CTAs of a persistent attend launch: one per item up to one per SM, or the test cap
+static int attend_grid(int n_items, int sms) {
+    int g = std::max(1, std::min(n_items, sms));
+    return t_attend_ctas > 0 ? std::min(g, t_attend_ctas) : g;
+}
 
 namespace veda {
 // The three device forms of 2^x, element by element (test hook for the attend kernel's exponentials).
@@ -513,8 +521,7 @@ static int launch_attend(DeviceState* ds, const AttendMaps& maps, const AttendAr
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_kernel)");
         ds->attend_attr[slot] = true;
     }
-    const int grid = std::max(1, std::min(a.n_items, ds->sms));
-    attend_kernel<D, kQK, kDirect><<<grid, C::kThreads, C::kSmem, s>>>(maps, a);
+    attend_kernel<D, kQK, kDirect><<<attend_grid(a.n_items, ds->sms), C::kThreads, C::kSmem, s>>>(maps, a);
     return launch_check("attend_kernel");
 }
 
@@ -630,7 +637,7 @@ static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, 
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_pair_kernel)");
         ds->pair_attr[slot] = true;
     }
-    attend_pair_kernel<D, kDirect><<<std::max(1, std::min(p.n_items, ds->sms)), C::kThreads, C::kSmem, s>>>(maps, p);
+    attend_pair_kernel<D, kDirect><<<attend_grid(p.n_items, ds->sms), C::kThreads, C::kSmem, s>>>(maps, p);
     if (int rc = launch_check("attend_pair_kernel")) return rc;
     // the redo pass over the listed items (at most n_items); CTAs past the list's length return at once
     a.redo_items = ws.redo_items;

@@ -56,7 +56,7 @@ def oracle_out(c, box, heads, res, q, k, v, want, idx=None, cnt=None):
 
 def redo_flags(lay, n, ws):
     """The redo flags the paired launch left in its workspace ([n, n_tiles] int32 after the merged lists and
-    their counts, each region 256-byte aligned), checked against the redo list that follows them: its
+    their counts (two int32 per pair), each region 256-byte aligned), checked against the redo list that follows them: its
     length (an int32 in a 256-byte slot) and its entries (single-tile item numbers: global query tiles
     first, head-major, then video ones)."""
     a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
@@ -259,3 +259,44 @@ def test_paired_malformed_lists_and_bad_arguments():
         L.veda_attend_paired(lay, res["q_t"], res["k_t"], res["v_t"], res["kept_idx"], res["kept_cnt"], out,
                              res["heads"], row_sq, max_sq, torch.empty(ws.numel() + 512, dtype=torch.uint8,
                                                                        device="cuda")[16:])
+
+
+@pytest.mark.parametrize("name", ["small_mixed", "small_d128", "padded_tiny"])
+@pytest.mark.parametrize("ctas", [1, 3])
+def test_many_items_per_cta(name, ctas):
+    # with the attend launches capped at 1 or 3 CTAs each CTA walks many pair items (and the single-tile
+    # kernel many query tiles) in a row, as every CTA does on a full-size layer: ring positions, barrier
+    # phases and the per-item state carry across items. Both paired entry points and both single-tile ones
+    # give the same output as with one CTA per item, bit for bit
+    c = case(name)
+    wl = c.wl
+    outs = {}
+    for cap in (0, ctas):
+        L.veda_debug_attend_ctas(cap)
+        try:
+            for kind in ("paired_direct", "paired", "direct", "tile"):
+                out = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+                for box, heads in c.groups:
+                    res = c.run_group(box, heads)
+                    lay = res["layout"]
+                    n = len(heads)
+                    row_sq, max_sq = norms(lay, c.dq, c.dk, res["heads"], n, wl.seq_len)
+                    ws = L.paired_workspace(lay, n)
+                    if kind == "paired_direct":
+                        L.veda_attend_direct_paired(lay, c.dq, c.dk, c.dv, res["kept_idx"], res["kept_cnt"], out,
+                                                    res["heads"], row_sq, max_sq, ws)
+                    elif kind == "paired":
+                        L.veda_attend_paired(lay, res["q_t"], res["k_t"], res["v_t"], res["kept_idx"], res["kept_cnt"],
+                                             out, res["heads"], row_sq, max_sq, ws)
+                    elif kind == "direct":
+                        L.veda_attend_direct(lay, c.dq, c.dk, c.dv, res["kept_idx"], res["kept_cnt"], out,
+                                             res["heads"], q_row_sq=row_sq, k_max_sq=max_sq)
+                    else:
+                        L.veda_attend(lay, res["q_t"], res["k_t"], res["v_t"], res["kept_idx"], res["kept_cnt"], out,
+                                      res["heads"], q_row_sq=row_sq, k_max_sq=max_sq)
+                    assert L.veda_sync_status() == L.VEDA_OK, (kind, cap, L.veda_last_error())
+                outs[(kind, cap)] = out
+        finally:
+            L.veda_debug_attend_ctas(0)
+    for kind in ("paired_direct", "paired", "direct", "tile"):
+        assert torch.equal(outs[(kind, 0)], outs[(kind, ctas)]), kind

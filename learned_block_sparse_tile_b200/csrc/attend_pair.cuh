@@ -28,8 +28,8 @@
 //   warps 4-19   two softmax groups of eight warps (units 0, 2, 4, ... and 1, 3, 5, ...), two threads per
 //                TMEM lane (key columns 0-63 and 64-127 of S), as in attend.cuh; each thread keeps the
 //                row sums of both query tiles. At the end of the item the four threads of a row add up
-//                the sums, group 0 writes query tile A and group 1 query tile B, each thread half of the
-//                row's columns.
+//                the sums (before the item's last PVs complete), group 0 writes query tile A and group 1
+//                query tile B, each thread half of the row's columns.
 // TMEM columns: S/P of group 0 [0,128), group 1 [128,256); O of query tile A [256, 256 + D), B [384, 384 + D).
 // Every wait is bounded (as in attend.cuh): on expiry the CTA drains, frees its TMEM and returns.
 #pragma once
@@ -224,12 +224,12 @@ struct PairCfg {
     static constexpr int kBoxes = D / 64;           // 128-byte-wide TMA boxes per tile
     static constexpr int kKStages = D == 128 ? 2 : 4;
     static constexpr int kVStages = D == 128 ? 2 : 4;
-    // header: barriers, then the end-of-item (sum A, sum B) of each [group][half][row]; then the
-    // 1024-aligned tiles (at head_dim 128: 197 KB of the 227 KB a CTA may use)
+    // header: barriers, then the end-of-item (sum A, sum B) of each [item parity][group][half][row]; then
+    // the 1024-aligned tiles (at head_dim 128: 201 KB of the 227 KB a CTA may use)
     static constexpr int kOffBar = 0;
     static constexpr int kOffStats = 512;
-    static constexpr int kHeader = 5120;
-    static_assert(kOffStats + 2 * 2 * 128 * 8 <= kHeader, "header layout");
+    static constexpr int kHeader = 9216;
+    static_assert(kOffStats + 2 * 2 * 2 * 128 * 8 <= kHeader, "header layout");
     static constexpr int kOffQ = kHeader;  // Q of tile A, then of tile B
     static constexpr int kOffK = kOffQ + 2 * kTileBytes;
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(640, 1)
     PairBars& B = *reinterpret_cast<PairBars*>(smem + C::kOffBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&B + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float2* stats = reinterpret_cast<float2*>(smem + C::kOffStats);  // [2 groups][2 halves][128 rows]
+    float2* stats = reinterpret_cast<float2*>(smem + C::kOffStats);  // [item parity][2 groups][2 halves][128 rows]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -608,21 +608,22 @@ __global__ void __launch_bounds__(640, 1)
                     sum_a = ptx::f2_add(sum_a, tot);
             }
             if (!ok) break;
-            ok = ptx::mbar_wait(&B.o_done, it & 1, abort_flag, tmo);  // every PV of the item is complete
             cu += nw;
-            if (!ok) break;
-            // the row sums of A and B: each thread publishes its part, then reads the row's four parts
+            // the row sums of A and B are final with the thread's last unit: each thread publishes its part
+            // and reads the row's four parts while the item's last PVs still run, so that after them only
+            // the read of O stands before its release. The sums of consecutive items use the two halves of
+            // the buffer: a thread can publish the next item's before every thread has read this one's
+            float2* st = stats + (it & 1) * 512;
             {
                 float a0, a1, b0, b1;
                 ptx::f2_unpack(sum_a, a0, a1);
                 ptx::f2_unpack(sum_b, b0, b1);
-                stats[(w * 2 + half) * 128 + row] = make_float2(a0 + a1, b0 + b1);
+                st[(w * 2 + half) * 128 + row] = make_float2(a0 + a1, b0 + b1);
             }
             ptx::mbar_arrive(&B.merge);
             ok = ptx::mbar_wait(&B.merge, it & 1, abort_flag, tmo);
-            ++it;
             if (!ok) break;
-            const float2 g00 = stats[row], g01 = stats[128 + row], g10 = stats[256 + row], g11 = stats[384 + row];
+            const float2 g00 = st[row], g01 = st[128 + row], g10 = st[256 + row], g11 = st[384 + row];
             const float l = w ? (g00.y + g01.y) + (g10.y + g11.y) : (g00.x + g01.x) + (g10.x + g11.x);
             const bool have = n_out > 0;
             // a real row whose sum left [2^-60, 2^100] (or is NaN): the exact redo rewrites its query tile
@@ -635,6 +636,9 @@ __global__ void __launch_bounds__(640, 1)
                 a.redo_items[atomicAdd(a.redo_count, 1)] = single;
             }
             const float inv = l > 0.f ? 1.f / l : 0.f;
+            ok = ptx::mbar_wait(&B.o_done, it & 1, abort_flag, tmo);  // every PV of the item is complete
+            ++it;
+            if (!ok) break;
             ptx::tc_fence_after();
             // this thread's half of the row is read (and scaled into bf16 pairs) before O is released to the
             // next item's first PV; the global stores come after the release

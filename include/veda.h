@@ -343,13 +343,14 @@ int veda_quantize_fp8(const veda_layout* layout, const void* x_t, int32_t n_head
 /* FP8 Q/K variant, steps 0 and 1 in one pass: veda_gather with the tile written as e4m3 codes and its
  * per-tile scale (the quantisation of veda_quantize_fp8, bit for bit) instead of bf16, so the bf16 tile
  * copy is never written or read back.
- *  x, x_strides, h_total, heads, feats  as veda_gather (feats may be NULL).
+ *  x, x_strides, h_total, heads, feats, row_sq, max_sq  as veda_gather (feats, row_sq and max_sq may be
+ *          NULL; the norms are those of the bf16 input, for the paired attend's logit bound).
  *  codes   device e4m3 bytes [n_heads, N, D] out (padding slots 0).
  *  scales  device fp32 [n_heads, n_tiles] out.
  * D must be 64 or 128. Errors as veda_gather. */
 int veda_gather_fp8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
                     int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales, float* feats,
-                    void* stream);
+                    float* row_sq, float* max_sq, void* stream);
 
 /* FP8 Q/K variant, step 2: veda_attend with Q and K given as e4m3 codes and per-tile scales (from
  * veda_quantize_fp8); S = Q K^T runs as an e4m3 x e4m3 tensor-core product with fp32 accumulation and is
@@ -374,13 +375,31 @@ int veda_attend_fp8(const veda_layout* layout, const void* q_codes, const void* 
  * veda_attend_int8: veda_attend on int8 codes and scales (arguments as veda_attend_fp8). D must be 128. */
 int veda_gather_int8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
                      int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales, float* feats,
-                     void* stream);
+                     float* row_sq, float* max_sq, void* stream);
 int veda_quantize_int8(const veda_layout* layout, const void* x_t, int32_t n_heads, int32_t dim, void* codes,
                        float* scales, void* stream);
 int veda_attend_int8(const veda_layout* layout, const void* q_codes, const void* k_codes, const float* scales_q,
                      const float* scales_k, const void* v_t, int32_t n_heads, int32_t dim, const int32_t* kept_idx,
                      const int32_t* kept_cnt, void* out, const int64_t out_strides[3], int32_t h_total,
                      const int32_t* heads, void* stream);
+
+/* The paired attend (see veda_attend_paired) on 8-bit Q/K codes: veda_attend_fp8 / veda_attend_int8's
+ * operation, two neighbouring query tiles per work item sharing each kept K/V tile load. Each row's softmax
+ * reference comes from the logit bound of the bf16 inputs (q_row_sq and k_max_sq from veda_gather_fp8 /
+ * veda_gather_int8 or veda_pool): the codes' logits differ from the bf16 ones only by the quantisation
+ * error, far inside the reference's 2^64 headroom, and a query tile the bound cannot serve is recomputed by
+ * veda_attend_fp8 / veda_attend_int8's kernel. Arguments as veda_attend_fp8 plus q_row_sq, k_max_sq,
+ * workspace and workspace_bytes as veda_attend_paired. D must be 128. */
+int veda_attend_fp8_paired(const veda_layout* layout, const void* q_codes, const void* k_codes,
+                           const float* scales_q, const float* scales_k, const void* v_t, int32_t n_heads,
+                           int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                           const int64_t out_strides[3], int32_t h_total, const int32_t* heads, const float* q_row_sq,
+                           const float* k_max_sq, void* workspace, size_t workspace_bytes, void* stream);
+int veda_attend_int8_paired(const veda_layout* layout, const void* q_codes, const void* k_codes,
+                            const float* scales_q, const float* scales_k, const void* v_t, int32_t n_heads,
+                            int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                            const int64_t out_strides[3], int32_t h_total, const int32_t* heads, const float* q_row_sq,
+                            const float* k_max_sq, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronizes `stream`, then reads and clears this device's latched kernel error word.
  * Returns VEDA_OK, VEDA_ERR_TIMEOUT, VEDA_ERR_BAD_LIST or VEDA_ERR_CUDA. */

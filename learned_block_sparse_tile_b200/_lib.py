@@ -25,6 +25,7 @@ EXPORTS = [
     "veda_quantize_int8", "veda_gather_int8", "veda_attend_int8", "veda_layout_export_direct", "veda_pool",
     "veda_attend_direct", "veda_debug_exp2", "veda_grid_of", "veda_describe_packed_layout",
     "veda_attend_paired_workspace_bytes", "veda_attend_paired", "veda_attend_direct_paired", "veda_debug_attend_ctas",
+    "veda_attend_fp8_paired", "veda_attend_int8_paired",
 ]
 
 VEDA_SEG_OTHER, VEDA_SEG_VIDEO, VEDA_SEG_COND, VEDA_SEG_REF_IMG = range(4)
@@ -110,11 +111,14 @@ def lib():
         L.veda_select.argtypes = [vp, p, i32, p, p, vp]
         L.veda_attend.argtypes = [vp, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, p, p, vp]
         L.veda_quantize_fp8.argtypes = [vp, p, i32, i32, p, p, vp]
-        L.veda_gather_fp8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
+        L.veda_gather_fp8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, p, p, vp]
         L.veda_quantize_int8.argtypes = [vp, p, i32, i32, p, p, vp]
-        L.veda_gather_int8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, vp]
+        L.veda_gather_int8.argtypes = [vp, p, C.POINTER(C.c_int64), i32, i32, p, i32, p, p, p, p, p, vp]
         L.veda_attend_fp8.argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
         L.veda_attend_int8.argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, vp]
+        for name in ("veda_attend_fp8_paired", "veda_attend_int8_paired"):
+            getattr(L, name).argtypes = [vp, p, p, p, p, p, i32, i32, p, p, p, C.POINTER(C.c_int64), i32, p, p, p, p,
+                                         C.c_size_t, vp]
         L.veda_sync_status.argtypes = [vp]
         L.veda_last_error.restype = C.c_char_p
         L.veda_set_wait_timeout_ns.argtypes = [C.c_uint64]
@@ -313,11 +317,12 @@ def veda_attend_direct_paired(layout, q, k, v, kept_idx, kept_cnt, out, heads, q
                                            workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
-def veda_gather_fp8(layout, x, heads, codes, scales, feats=None, stream=None):
+def veda_gather_fp8(layout, x, heads, codes, scales, feats=None, stream=None, row_sq=None, max_sq=None):
     """x: bf16 [S, H, D] cuda; heads: int32 [n] cuda; codes: uint8 [n, N, D] (e4m3 bytes); scales: fp32
-    [n, n_tiles]; feats: fp32 [n, n_video, 3D] or None."""
+    [n, n_tiles]; feats: fp32 [n, n_video, 3D] or None; row_sq / max_sq: the bf16 norms (as veda_gather)."""
     _check(lib().veda_gather_fp8(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
-                                 heads.numel(), _ptr(codes), _ptr(scales), _ptr(feats), _stream(stream)))
+                                 heads.numel(), _ptr(codes), _ptr(scales), _ptr(feats), _ptr(row_sq), _ptr(max_sq),
+                                 _stream(stream)))
 
 
 def veda_quantize_fp8(layout, x_t, codes, scales, stream=None):
@@ -333,10 +338,11 @@ def veda_attend_fp8(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx,
                                  _strides(out), out.shape[1], _ptr(heads), _stream(stream)))
 
 
-def veda_gather_int8(layout, x, heads, codes, scales, feats=None, stream=None):
+def veda_gather_int8(layout, x, heads, codes, scales, feats=None, stream=None, row_sq=None, max_sq=None):
     """veda_gather_fp8 with int8 codes (int8 or uint8 [n, N, D])."""
     _check(lib().veda_gather_int8(layout.handle, _ptr(x), _strides(x), x.shape[1], x.shape[2], _ptr(heads),
-                                  heads.numel(), _ptr(codes), _ptr(scales), _ptr(feats), _stream(stream)))
+                                  heads.numel(), _ptr(codes), _ptr(scales), _ptr(feats), _ptr(row_sq), _ptr(max_sq),
+                                  _stream(stream)))
 
 
 def veda_quantize_int8(layout, x_t, codes, scales, stream=None):
@@ -350,6 +356,29 @@ def veda_attend_int8(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx
     _check(lib().veda_attend_int8(layout.handle, _ptr(q_codes), _ptr(k_codes), _ptr(scales_q), _ptr(scales_k),
                                   _ptr(v_t), v_t.shape[0], v_t.shape[2], _ptr(kept_idx), _ptr(kept_cnt), _ptr(out),
                                   _strides(out), out.shape[1], _ptr(heads), _stream(stream)))
+
+
+def _attend_codes_paired(fn, layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx, kept_cnt, out, heads,
+                         q_row_sq, k_max_sq, workspace, stream):
+    _check(fn(layout.handle, _ptr(q_codes), _ptr(k_codes), _ptr(scales_q), _ptr(scales_k), _ptr(v_t), v_t.shape[0],
+              v_t.shape[2], _ptr(kept_idx), _ptr(kept_cnt), _ptr(out), _strides(out), out.shape[1], _ptr(heads),
+              _ptr(q_row_sq), _ptr(k_max_sq), _ptr(workspace), workspace.numel() * workspace.element_size(),
+              _stream(stream)))
+
+
+def veda_attend_fp8_paired(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx, kept_cnt, out, heads,
+                           q_row_sq, k_max_sq, workspace, stream=None):
+    """veda_attend_fp8 two neighbouring query tiles at a time (as veda_attend_paired; the norms of the bf16
+    inputs from veda_gather_fp8, workspace from paired_workspace)."""
+    _attend_codes_paired(lib().veda_attend_fp8_paired, layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx,
+                         kept_cnt, out, heads, q_row_sq, k_max_sq, workspace, stream)
+
+
+def veda_attend_int8_paired(layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx, kept_cnt, out, heads,
+                            q_row_sq, k_max_sq, workspace, stream=None):
+    """veda_attend_int8 two neighbouring query tiles at a time (as veda_attend_fp8_paired)."""
+    _attend_codes_paired(lib().veda_attend_int8_paired, layout, q_codes, k_codes, scales_q, scales_k, v_t, kept_idx,
+                         kept_cnt, out, heads, q_row_sq, k_max_sq, workspace, stream)
 
 
 def veda_sync_status(stream=None):

@@ -1,5 +1,7 @@
 // Block-sparse flash attention over kept 128x128 tiles for two neighbouring query tiles at once, sm_100a
-// (tcgen05 + TMA), bf16 Q/K/V with the logit bound. Same operation as attend.cuh (veda_core.py
+// (tcgen05 + TMA), with the logit bound; Q/K in bf16 or as 8-bit codes with per-tile scales (e4m3 or int8,
+// as attend.cuh's 8-bit variants: S = Q K^T on the kind::f8f6f4 / kind::i8 path, times both tiles' scales),
+// V in bf16. Same operation as attend.cuh (veda_core.py
 // (ComfyUI-FunPack), "selection", reference_attend, then "tiles", scatter_): for query tile i of head h,
 // softmax(q k^T * D^-0.5) v over the real key slots of its kept tiles, 0 for a row that sees no key.
 //
@@ -160,6 +162,8 @@ struct PairArgs {
     const int4* tile_coord;  // gather-free variant, as in AttendArgs
     const uint4* tile_mask;
     int32_t n_map_spans;
+    const float* scales_q;  // 8-bit variants: [n_heads, n_tiles] per-tile scales of the Q and K codes
+    const float* scales_k;
     const float* q_row_sq;  // [n_heads, seq_len]
     const float* k_max_sq;  // [n_heads]
     int64_t seq_len;
@@ -215,28 +219,34 @@ __device__ __forceinline__ int32_t item_unit(const PairArgs& a, const PairItem& 
     return a.units[it.pair * (2 * int64_t(a.max_kept)) + j];
 }
 
-template <int D>
+template <int D, int kQK = kQKBf16>
 struct PairCfg {
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static constexpr bool kFp8 = kQK != kQKBf16;  // Q and K are 8-bit codes with per-tile scales
+    static_assert(!kFp8 || D == 128, "the 8-bit Q/K variants are built for head_dim 128");
     static constexpr int kWarps = 20;
     static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kTileBytes = 128 * D * 2;  // one Q, K or V tile
-    static constexpr int kBoxes = D / 64;           // 128-byte-wide TMA boxes per tile
-    static constexpr int kKStages = D == 128 ? 2 : 4;
-    static constexpr int kVStages = D == 128 ? 2 : 4;
+    static constexpr int kQKBytes = 128 * D * (kFp8 ? 1 : 2);  // one Q or K tile
+    static constexpr int kTileBytes = 128 * D * 2;             // one V tile (bf16)
+    static constexpr int kBoxesQK = kFp8 ? 1 : D / 64;         // 128-byte-wide TMA boxes per Q or K tile
+    static constexpr int kBoxes = D / 64;                      // 128-byte-wide TMA boxes per V tile
+    static constexpr int kKStages = kFp8 ? 4 : (D == 128 ? 2 : 4);
+    static constexpr int kVStages = kFp8 ? 3 : (D == 128 ? 2 : 4);
     // header: barriers, then the end-of-item (sum A, sum B) of each [item parity][group][half][row]; then
-    // the 1024-aligned tiles (at head_dim 128: 201 KB of the 227 KB a CTA may use)
+    // the 1024-aligned tiles (201 KB of the 227 KB a CTA may use at head_dim 128, either format)
     static constexpr int kOffBar = 0;
     static constexpr int kOffStats = 512;
     static constexpr int kHeader = 9216;
     static_assert(kOffStats + 2 * 2 * 2 * 128 * 8 <= kHeader, "header layout");
     static constexpr int kOffQ = kHeader;  // Q of tile A, then of tile B
-    static constexpr int kOffK = kOffQ + 2 * kTileBytes;
-    static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+    static constexpr int kOffK = kOffQ + 2 * kQKBytes;
+    static constexpr int kOffV = kOffK + kKStages * kQKBytes;
     static constexpr int kSmem = kOffV + kVStages * kTileBytes;
     static_assert(kSmem <= 227 * 1024, "shared memory");
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, false, false);
+    static constexpr uint32_t kIdescS = kQK == kQKI8    ? ptx::idesc_s8_s32(128, 128)
+                                        : kQK == kQKE4M3 ? ptx::idesc_e4m3_f32(128, 128)
+                                                         : ptx::idesc_bf16_f32(128, 128, false, false);
     static constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, false, true);
 };
 
@@ -247,10 +257,12 @@ struct PairBars {
     uint64_t o_done, o_empty, merge, drain;
 };
 
-template <int D, bool kDirect>
+template <int D, int kQK, bool kDirect>
 __global__ void __launch_bounds__(640, 1)
     attend_pair_kernel(const __grid_constant__ AttendMaps maps, const PairArgs a) {
-    using C = PairCfg<D>;
+    using C = PairCfg<D, kQK>;
+    constexpr bool kFp8 = C::kFp8;
+    static_assert(!(kFp8 && kDirect), "the 8-bit Q/K codes are tile-ordered copies");
     constexpr int KS = C::kKStages, VS = C::kVStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = smem_raw;
@@ -325,10 +337,10 @@ __global__ void __launch_bounds__(640, 1)
                 __all_sync(0xffffffffu, ptx::mbar_wait(&B.q_empty, (issued_q & 1) ^ 1, abort_flag, tmo))) {
                 if (ptx::elect_one()) {
                     const int nq = pi.qb >= 0 ? 2 : 1;
-                    ptx::mbar_arrive_expect_tx(&B.q_full, nq * C::kTileBytes);
+                    ptx::mbar_arrive_expect_tx(&B.q_full, nq * C::kQKBytes);
                     for (int x = 0; x < nq; ++x) {
                         const int qt = x ? pi.qb : pi.qa;
-                        uint8_t* dst = smem + C::kOffQ + x * C::kTileBytes;
+                        uint8_t* dst = smem + C::kOffQ + x * C::kQKBytes;
                         if constexpr (kDirect) {
                             const int4 tc = __ldg(a.tile_coord + qt);
                             for (int b = 0; b < C::kBoxes; ++b) {
@@ -340,8 +352,9 @@ __global__ void __launch_bounds__(640, 1)
                                                           &B.q_full, keep);
                             }
                         } else {
-                            for (int b = 0; b < C::kBoxes; ++b)
-                                ptx::tma_load_2d(dst + b * 16384, &maps.q[0], b * 64, row0 + qt * 128, &B.q_full);
+                            for (int b = 0; b < C::kBoxesQK; ++b)
+                                ptx::tma_load_2d(dst + b * 16384, &maps.q[0], b * (kFp8 ? 128 : 64), row0 + qt * 128,
+                                                 &B.q_full);
                         }
                     }
                 }
@@ -369,11 +382,13 @@ __global__ void __launch_bounds__(640, 1)
                 const int st = issued % S, ph = issued / S;
                 uint64_t* empty = kq ? &B.k_empty[st] : &B.v_empty[st];
                 uint64_t* full = kq ? &B.k_full[st] : &B.v_full[st];
-                uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * C::kTileBytes;
+                const int bytes = kq ? C::kQKBytes : C::kTileBytes;
+                uint8_t* dst = smem + (kq ? C::kOffK : C::kOffV) + st * bytes;
                 if (__all_sync(0xffffffffu, ptx::mbar_wait(empty, (ph & 1) ^ 1, abort_flag, tmo))) {
                     if (ptx::elect_one()) {
-                        ptx::mbar_arrive_expect_tx(full, C::kTileBytes);
-                        for (int b = 0; b < C::kBoxes; ++b) {
+                        ptx::mbar_arrive_expect_tx(full, bytes);
+                        const int boxes = kq ? C::kBoxesQK : C::kBoxes, xstep = (kq && kFp8) ? 128 : 64;
+                        for (int b = 0; b < boxes; ++b) {
                             if constexpr (kDirect) {
                                 if (tc.x >= 0)
                                     ptx::tma_load_5d_hint(dst + b * 16384, kq ? &maps.k[tc.x] : &maps.v[tc.x], b * 64, head,
@@ -383,7 +398,7 @@ __global__ void __launch_bounds__(640, 1)
                                                           kq ? &maps.k[kGlobalMapSet] : &maps.v[kGlobalMapSet], b * 64,
                                                           head, tc.y, full, keep);
                             } else {
-                                ptx::tma_load_2d_hint(dst + b * 16384, kq ? &maps.k[0] : &maps.v[0], b * 64, y, full,
+                                ptx::tma_load_2d_hint(dst + b * 16384, kq ? &maps.k[0] : &maps.v[0], b * xstep, y, full,
                                                       keep);
                             }
                         }
@@ -459,12 +474,25 @@ __global__ void __launch_bounds__(640, 1)
                         if ((us & 2) && !__all_sync(0xffffffffu, ptx::mbar_wait(&B.k_full[ks], kph, abort_flag, tmo)))
                             return false;
                         ptx::tc_fence_after();
-                        const uint64_t dks = dk + uint64_t(ks * (C::kTileBytes >> 4));
-                        const uint64_t dqx = dq + uint64_t((us & 1) * (C::kTileBytes >> 4));
+                        const uint64_t dks = dk + uint64_t(ks * (C::kQKBytes >> 4));
+                        const uint64_t dqx = dq + uint64_t((us & 1) * (C::kQKBytes >> 4));
+                        if constexpr (kFp8) {
+                            // 8-bit codes: one 128-byte box holds the tile's 128 columns, 32 per k-step
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t off = uint64_t((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
-                            ptx::mma_bf16_ss_w(tmem + 128 * w, dqx + off, dks + off, C::kIdescS, kk > 0);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                if constexpr (kQK == kQKI8)
+                                    ptx::mma_i8_ss_w(tmem + 128 * w, dqx + uint64_t(kk * 2), dks + uint64_t(kk * 2),
+                                                     C::kIdescS, kk > 0);
+                                else
+                                    ptx::mma_f8_ss_w(tmem + 128 * w, dqx + uint64_t(kk * 2), dks + uint64_t(kk * 2),
+                                                     C::kIdescS, kk > 0);
+                            }
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint64_t off = uint64_t((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
+                                ptx::mma_bf16_ss_w(tmem + 128 * w, dqx + off, dks + off, C::kIdescS, kk > 0);
+                            }
                         }
                         ptx::mma_commit_w(&B.s_full[w]);
                         if (us & 4) {  // the key tile's last S: its K slot may be refilled once it completes
@@ -507,7 +535,6 @@ __global__ void __launch_bounds__(640, 1)
         const uint32_t t_s = tmem + lane_base + 128 * w + 64 * half;  // this half's S columns (its P: the first 32)
         constexpr int kCols = D / 2;                                  // output columns each thread writes
         const uint32_t t_o = tmem + lane_base + 256 + 128 * w + half * kCols;
-        const uint64_t sl2x2 = ptx::f2_pack(a.scale_log2, a.scale_log2);
         int cu = 0;  // units this group has had so far (barrier phases)
         int it = 0;  // items with units so far
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
@@ -540,18 +567,28 @@ __global__ void __launch_bounds__(640, 1)
                 return kBoundOffset - bound;
             };
             const float negm_a = neg_ref(prow_a), negm_b = neg_ref(prow_b);
+            // 8-bit codes: the query tiles' scales (the key tiles' come with their units)
+            const float sq_a = kFp8 ? __ldg(a.scales_q + int64_t(pi.hh) * a.n_tiles + pi.qa) : 1.f;
+            const float sq_b = kFp8 && pi.qb >= 0 ? __ldg(a.scales_q + int64_t(pi.hh) * a.n_tiles + pi.qb) : 1.f;
             uint64_t sum_a = ptx::f2_pack(0.f, 0.f), sum_b = ptx::f2_pack(0.f, 0.f);
             bool ok = true;
             int my_unit = 0, my_vc = 128;
+            float my_sk = 1.f;
             const int nw = group_tiles(n, w);
             for (int k = 0; k < nw; ++k) {
                 if ((k & 31) == 0) {
                     const int jj = 2 * (k + lane) + w;
                     my_unit = jj < n ? item_unit(a, pi, jj) : 0;
                     my_vc = jj < n ? __ldg(a.valid_count + (my_unit >> 3)) : 128;
+                    if (kFp8) my_sk = jj < n ? __ldg(a.scales_k + int64_t(pi.hh) * a.n_tiles + (my_unit >> 3)) : 1.f;
                 }
                 const int u = __shfl_sync(0xffffffffu, my_unit, k & 31);
                 const int vc = __shfl_sync(0xffffffffu, my_vc, k & 31);
+                // log2-domain scale of this unit's logits (the 8-bit codes also undo both tiles' scales)
+                const float sl2 =
+                    kFp8 ? a.scale_log2 * (((u & 1) ? sq_b : sq_a) * __shfl_sync(0xffffffffu, my_sk, k & 31))
+                         : a.scale_log2;
+                const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
                 ok = ptx::mbar_wait(&B.s_full[w], (cu + k) & 1, abort_flag, tmo);
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -561,6 +598,19 @@ __global__ void __launch_bounds__(640, 1)
                 ptx::tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(s));
                 ptx::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
                 ptx::tmem_wait_ld();
+                if constexpr (kQK == kQKI8) {
+                    // int32 -> fp32, exactly: adding the bit pattern of 1.5 * 2^23 puts |S| < 2^22 in the
+                    // low mantissa bits of a float in [2^23, 2^24); subtracting 1.5 * 2^23 is then exact
+                    const uint64_t magic = ptx::f2_pack(-12582912.f, -12582912.f);
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        float f0, f1;
+                        ptx::f2_unpack(ptx::f2_add(ptx::f2_pack(__uint_as_float(s[c] + 0x4B400000u),
+                                                                __uint_as_float(s[c + 1] + 0x4B400000u)), magic), f0, f1);
+                        s[c] = __float_as_uint(f0);
+                        s[c + 1] = __float_as_uint(f1);
+                    }
+                }
                 if (vc < 128) {
                     if constexpr (kDirect) {
                         const uint4 m = __ldg(a.tile_mask + (u >> 3));

@@ -37,7 +37,7 @@ struct DeviceState {
     int sms = 0;
     int* err = nullptr;  // device address of g_err
     bool attend_attr[8] = {};  // (head_dim 128) + 2 * Q/K format; 6 + (head_dim 128) for the gather-free variant
-    bool pair_attr[4] = {};    // paired kernel: (head_dim 128) + 2 * gather-free
+    bool pair_attr[12] = {};   // paired kernel: (head_dim 128) + 2 * gather-free + 4 * Q/K format
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -328,13 +328,14 @@ extern "C" int veda_pool(const veda_layout* layout, const void* x, const int64_t
 // veda_gather_fp8 / veda_gather_int8: the gather writing 8-bit codes and per-tile scales.
 static int gather_codes(const char* who, int code, const veda_layout* layout, const void* x,
                         const int64_t x_strides[3], int32_t h_total, int32_t dim, const int32_t* heads, int32_t n_heads,
-                        void* codes, float* scales, float* feats, void* stream) {
+                        void* codes, float* scales, float* feats, float* row_sq, float* max_sq, void* stream) {
     clear_error();
     if (!layout || !x || !heads || !codes || !scales) return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
     if (dim != 64 && dim != 128) return fail(VEDA_ERR_INVALID, std::string(who) + ": head_dim must be 64 or 128");
     if (n_heads <= 0 || h_total <= 0) return fail(VEDA_ERR_INVALID, std::string(who) + ": head counts must be positive");
     if (int rc = check_strided(x_strides, x, who)) return rc;
-    if (!aligned16(codes) || !aligned16(scales) || (feats && !aligned16(feats)))
+    if (!aligned16(codes) || !aligned16(scales) || (feats && !aligned16(feats)) || (row_sq && !aligned16(row_sq)) ||
+        (max_sq && !aligned16(max_sq)))
         return fail(VEDA_ERR_INVALID, std::string(who) + ": outputs need 16-byte alignment");
     DeviceState* ds;
     if (int rc = device_state(&ds)) return rc;
@@ -357,11 +358,12 @@ static int gather_codes(const char* who, int code, const veda_layout* layout, co
     a.n_video = d.n_video;
     a.h_total = h_total;
     a.err = ds->err;
-    a.row_sq = nullptr;
-    a.max_sq = nullptr;
+    a.row_sq = row_sq;
+    a.max_sq = reinterpret_cast<unsigned*>(max_sq);
     a.seq_len = d.seq_len;
     dim3 grid(unsigned(d.n_tiles), unsigned(n_heads));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (int rc = clear_max_sq(max_sq, n_heads, s)) return rc;
     if (code == kCodeI8) {
         if (dim == 128)
             gather_pool_kernel<128, kCodeI8><<<grid, 256, 0, s>>>(a);
@@ -378,16 +380,16 @@ static int gather_codes(const char* who, int code, const veda_layout* layout, co
 
 extern "C" int veda_gather_fp8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
                                int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales,
-                               float* feats, void* stream) {
+                               float* feats, float* row_sq, float* max_sq, void* stream) {
     return gather_codes("veda_gather_fp8", kCodeE4M3, layout, x, x_strides, h_total, dim, heads, n_heads, codes,
-                        scales, feats, stream);
+                        scales, feats, row_sq, max_sq, stream);
 }
 
 extern "C" int veda_gather_int8(const veda_layout* layout, const void* x, const int64_t x_strides[3], int32_t h_total,
                                 int32_t dim, const int32_t* heads, int32_t n_heads, void* codes, float* scales,
-                                float* feats, void* stream) {
+                                float* feats, float* row_sq, float* max_sq, void* stream) {
     return gather_codes("veda_gather_int8", kCodeI8, layout, x, x_strides, h_total, dim, heads, n_heads, codes,
-                        scales, feats, stream);
+                        scales, feats, row_sq, max_sq, stream);
 }
 
 extern "C" size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim) {
@@ -563,7 +565,7 @@ extern "C" size_t veda_attend_paired_workspace_bytes(const veda_layout* layout, 
 
 // The paired attend: clear the redo flags, merge each pair's lists into units, run the paired kernel, then
 // the single-tile kernel over the query tiles it flagged (an empty pass when none is).
-template <int D, bool kDirect>
+template <int D, int kQK, bool kDirect>
 static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, const int32_t* kept_idx,
                          const int32_t* kept_cnt, void* workspace, cudaStream_t s) {
     const PairWorkspace ws = pair_workspace(a.n_video, a.max_kept, a.n_tiles, a.n_heads, workspace);
@@ -624,26 +626,29 @@ static int launch_paired(DeviceState* ds, const AttendMaps& maps, AttendArgs a, 
     p.tile_coord = a.tile_coord;
     p.tile_mask = a.tile_mask;
     p.n_map_spans = a.n_map_spans;
+    p.scales_q = a.scales_q;
+    p.scales_k = a.scales_k;
     p.q_row_sq = a.q_row_sq;
     p.k_max_sq = a.k_max_sq;
     p.seq_len = a.seq_len;
     p.redo_flags = ws.flags;
     p.redo_items = ws.redo_items;
     p.redo_count = ws.redo_count;
-    using C = PairCfg<D>;
-    const int slot = (D == 128) + 2 * kDirect;
+    using C = PairCfg<D, kQK>;
+    const int slot = (D == 128) + 2 * kDirect + 4 * kQK;
     if (!ds->pair_attr[slot]) {
-        e = cudaFuncSetAttribute(attend_pair_kernel<D, kDirect>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        e = cudaFuncSetAttribute(attend_pair_kernel<D, kQK, kDirect>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attend_pair_kernel)");
         ds->pair_attr[slot] = true;
     }
-    attend_pair_kernel<D, kDirect><<<attend_grid(p.n_items, ds->sms), C::kThreads, C::kSmem, s>>>(maps, p);
+    attend_pair_kernel<D, kQK, kDirect><<<attend_grid(p.n_items, ds->sms), C::kThreads, C::kSmem, s>>>(maps, p);
     if (int rc = launch_check("attend_pair_kernel")) return rc;
     // the redo pass over the listed items (at most n_items); CTAs past the list's length return at once
     a.redo_items = ws.redo_items;
     a.redo_count = ws.redo_count;
     a.hold_q = 0;
-    return launch_attend<D, kQKBf16, kDirect>(ds, maps, a, s);
+    return launch_attend<D, kQK, kDirect>(ds, maps, a, s);
 }
 
 // The launch arguments both attend entry points share: lists, layout tables, output, limits and the wait
@@ -693,7 +698,10 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
                          const int32_t* heads, void* stream, int qk, const float* q_row_sq = nullptr,
                          const float* k_max_sq = nullptr, void* pair_ws = nullptr) {
     const bool fp8 = qk != kQKBf16;  // 8-bit Q/K codes (e4m3 or int8)
-    const char* who = qk == kQKI8 ? "veda_attend_int8" : fp8 ? "veda_attend_fp8" : pair_ws ? "veda_attend_paired" : "veda_attend";
+    const char* who = qk == kQKI8 ? (pair_ws ? "veda_attend_int8_paired" : "veda_attend_int8")
+                      : fp8       ? (pair_ws ? "veda_attend_fp8_paired" : "veda_attend_fp8")
+                      : pair_ws   ? "veda_attend_paired"
+                                  : "veda_attend";
     if (!layout || !q || !k || !v_t || !kept_idx || !kept_cnt || !out || !heads || (fp8 && (!sq || !sk)))
         return fail(VEDA_ERR_INVALID, std::string(who) + ": NULL argument");
     if (fp8 ? dim != 128 : (dim != 64 && dim != 128))
@@ -723,9 +731,16 @@ static int attend_common(const veda_layout* layout, const void* q, const void* k
         a.k_max_sq = k_max_sq;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (pair_ws)
-        return dim == 128 ? launch_paired<128, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s)
-                          : launch_paired<64, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
+    if (pair_ws) {
+        // the logit bound for the 8-bit codes comes from the bf16 norms: the codes' logits differ from the
+        // bf16 ones by the quantisation error, far inside the reference's 2^64 headroom
+        a.q_row_sq = q_row_sq;
+        a.k_max_sq = k_max_sq;
+        if (qk == kQKI8) return launch_paired<128, kQKI8, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
+        if (qk == kQKE4M3) return launch_paired<128, kQKE4M3, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
+        return dim == 128 ? launch_paired<128, kQKBf16, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s)
+                          : launch_paired<64, kQKBf16, false>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
+    }
     if (qk == kQKI8) return launch_attend<128, kQKI8>(ds, maps, a, s);
     if (qk == kQKE4M3) return launch_attend<128, kQKE4M3>(ds, maps, a, s);
     return dim == 128 ? launch_attend<128, kQKBf16>(ds, maps, a, s) : launch_attend<64, kQKBf16>(ds, maps, a, s);
@@ -854,8 +869,8 @@ static int attend_direct_impl(const veda_layout* layout, const void* q, const in
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (pair_ws)
-        return dim == 128 ? launch_paired<128, true>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s)
-                          : launch_paired<64, true>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
+        return dim == 128 ? launch_paired<128, kQKBf16, true>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s)
+                          : launch_paired<64, kQKBf16, true>(ds, maps, a, kept_idx, kept_cnt, pair_ws, s);
     return dim == 128 ? launch_attend<128, kQKBf16, true>(ds, maps, a, s) : launch_attend<64, kQKBf16, true>(ds, maps, a, s);
 }
 
@@ -901,6 +916,34 @@ extern "C" int veda_attend_int8(const veda_layout* layout, const void* q_codes, 
     clear_error();
     return attend_common(layout, q_codes, k_codes, scales_q, scales_k, v_t, n_heads, dim, kept_idx, kept_cnt, out,
                          out_strides, h_total, heads, stream, kQKI8);
+}
+
+extern "C" int veda_attend_fp8_paired(const veda_layout* layout, const void* q_codes, const void* k_codes,
+                                      const float* scales_q, const float* scales_k, const void* v_t, int32_t n_heads,
+                                      int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                                      const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
+                                      const float* q_row_sq, const float* k_max_sq, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+    clear_error();
+    if (int rc = check_paired("veda_attend_fp8_paired", layout, n_heads, q_row_sq, k_max_sq, workspace,
+                              workspace_bytes))
+        return rc;
+    return attend_common(layout, q_codes, k_codes, scales_q, scales_k, v_t, n_heads, dim, kept_idx, kept_cnt, out,
+                         out_strides, h_total, heads, stream, kQKE4M3, q_row_sq, k_max_sq, workspace);
+}
+
+extern "C" int veda_attend_int8_paired(const veda_layout* layout, const void* q_codes, const void* k_codes,
+                                       const float* scales_q, const float* scales_k, const void* v_t, int32_t n_heads,
+                                       int32_t dim, const int32_t* kept_idx, const int32_t* kept_cnt, void* out,
+                                       const int64_t out_strides[3], int32_t h_total, const int32_t* heads,
+                                       const float* q_row_sq, const float* k_max_sq, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+    clear_error();
+    if (int rc = check_paired("veda_attend_int8_paired", layout, n_heads, q_row_sq, k_max_sq, workspace,
+                              workspace_bytes))
+        return rc;
+    return attend_common(layout, q_codes, k_codes, scales_q, scales_k, v_t, n_heads, dim, kept_idx, kept_cnt, out,
+                         out_strides, h_total, heads, stream, kQKI8, q_row_sq, k_max_sq, workspace);
 }
 
 static int quantize_codes(const char* who, int code, const veda_layout* layout, const void* x_t, int32_t n_heads,

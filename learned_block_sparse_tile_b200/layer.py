@@ -26,13 +26,15 @@ class VedaLayer:
                  tile-order copies). None (default): used when Q/K are bf16 and every group's layout has a
                  box form (veda_layout_export_direct); True: required (raises otherwise); False: the
                  tile-order path (veda_gather + veda_attend), which takes every layout
-    logit_bound  bf16 paths: the pool/gather of Q also writes ||q||^2 per row and that of K the largest
-                 ||k||^2 per head, and the attend takes them as its logit bound (later tiles of an item may
-                 then skip the row max; same softmax). Default True; the 8-bit paths ignore it
-    paired       with the logit bound: the paired attend (veda_attend_paired / veda_attend_direct_paired),
-                 two neighbouring query tiles per work item sharing each kept K/V tile load, the softmax
-                 reference fixed by the bound, and an exact redo of any query tile the bound cannot serve.
-                 Default True; False keeps the single-tile attend
+    logit_bound  the pool/gather of Q also writes ||q||^2 per row and that of K the largest ||k||^2 per
+                 head, and the attend takes them as its logit bound (the single bf16 attend may then skip
+                 the row max on an item's later tiles; the paired attend takes its softmax reference from
+                 it; same softmax). Default True
+    paired       with the logit bound: the paired attend (veda_attend_paired / veda_attend_direct_paired,
+                 veda_attend_fp8_paired / veda_attend_int8_paired for the 8-bit Q/K), two neighbouring query
+                 tiles per work item sharing each kept K/V tile load, the softmax reference fixed by the
+                 bound, and an exact redo of any query tile the bound cannot serve. Default True; False
+                 keeps the single-tile attend
     """
 
     LAUNCHES_PER_GROUP = 7  # tile-order path: gather q, gather k, 2 score GEMMs, select, gather v, attend
@@ -62,8 +64,10 @@ class VedaLayer:
                 if not L.veda_layout_has_box_form(x):
                     L.veda_layout_export_direct(x)  # raises with the reason
         self.direct = bool(direct)
-        self.logit_bound = bool(logit_bound) and not (self.fp8_qk or self.int8_qk)
+        self.logit_bound = bool(logit_bound)
         self.paired = bool(paired) and self.logit_bound
+        # the 8-bit single-tile attend keeps exact per-tile maxima: its norms are needed only when paired
+        norms = self.logit_bound and (self.paired or not (self.fp8_qk or self.int8_qk))
         self.groups = []
         for box in sorted(groups):
             lay = layouts[box]
@@ -90,7 +94,7 @@ class VedaLayer:
                          k_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
             if not self.direct:
                 g.update(v_t=torch.empty(n, lay.n_slots, dim, dtype=torch.bfloat16, device=dev))
-            if self.logit_bound:
+            if norms:
                 g.update(q_row_sq=torch.empty(n, self.seq_len, dtype=torch.float32, device=dev),
                          k_max_sq=torch.empty(n, dtype=torch.float32, device=dev))
             else:
@@ -183,8 +187,8 @@ class VedaLayer:
             m = mark("gather_qk", st)
             if self.fp8_qk or self.int8_qk:
                 gather = L.veda_gather_int8 if self.int8_qk else L.veda_gather_fp8
-                gather(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st)
-                gather(lay, k, g["heads"], g["k8"], g["sk"], g["feats_k"], st)
+                gather(lay, q, g["heads"], g["q8"], g["sq"], g["feats_q"], st, row_sq=g["q_row_sq"])
+                gather(lay, k, g["heads"], g["k8"], g["sk"], g["feats_k"], st, max_sq=g["k_max_sq"])
             else:
                 L.veda_gather(lay, q, g["heads"], g["q_t"], g["feats_q"], st, row_sq=g["q_row_sq"])
                 L.veda_gather(lay, k, g["heads"], g["k_t"], g["feats_k"], st, max_sq=g["k_max_sq"])
@@ -205,7 +209,11 @@ class VedaLayer:
             done(m, st)
             st.wait_event(v_done)
             m = mark("attend", st)
-            if self.fp8_qk or self.int8_qk:
+            if (self.fp8_qk or self.int8_qk) and self.paired:
+                attend = L.veda_attend_int8_paired if self.int8_qk else L.veda_attend_fp8_paired
+                attend(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"],
+                       g["q_row_sq"], g["k_max_sq"], g["pair_ws"], st)
+            elif self.fp8_qk or self.int8_qk:
                 attend = L.veda_attend_int8 if self.int8_qk else L.veda_attend_fp8
                 attend(lay, g["q8"], g["k8"], g["sq"], g["sk"], g["v_t"], g["kept_idx"], g["kept_cnt"], out, g["heads"], st)
             elif self.paired:

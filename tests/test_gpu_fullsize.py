@@ -52,7 +52,7 @@ def test_full_size_layer(name, direct, paired):
     layer = VedaLayer(wl.seq_len, wl.ref_spans, wl.target, wl.head_shapes, (wl.generated, wl.reference),
                       wl.heads, wl.dim, fp8_qk=wl.fp8_qk, int8_qk=wl.int8_qk, direct=direct, paired=paired)
     assert layer.direct == (direct is None and not (wl.fp8_qk or wl.int8_qk))
-    assert layer.paired == (paired and not (wl.fp8_qk or wl.int8_qk))
+    assert layer.paired == paired
     layer.set_projections(x["pq"], x["pk"])
     out = torch.full_like(x["dq"], 7.0)
     layer.forward(x["dq"], x["dk"], x["dv"], out)

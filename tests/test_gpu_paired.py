@@ -300,3 +300,51 @@ def test_many_items_per_cta(name, ctas):
             L.veda_debug_attend_ctas(0)
     for kind in ("paired_direct", "paired", "direct", "tile"):
         assert torch.equal(outs[(kind, 0)], outs[(kind, ctas)]), kind
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("q_scale", [1.0, 16.0])
+def test_paired_8bit_codes(fmt, q_scale):
+    # veda_attend_fp8_paired / veda_attend_int8_paired against the oracle's 8-bit readings (bf16 tolerance)
+    # on the codes of the fused 8-bit gathers, which also write the norms of the bf16 inputs (equal to
+    # veda_pool's, bit for bit); q_scale 16 sends most query tiles to the exact redo. The result equals the
+    # single-tile 8-bit attend's within rounding
+    c = case("small_d128")
+    wl = c.wl
+    qs = c.dq * q_scale
+    q, k, v = f32(qs), f32(c.k), f32(c.v)
+    code_t = torch.int8 if fmt == "int8" else torch.uint8
+    gather = L.veda_gather_int8 if fmt == "int8" else L.veda_gather_fp8
+    paired = L.veda_attend_int8_paired if fmt == "int8" else L.veda_attend_fp8_paired
+    single = L.veda_attend_int8 if fmt == "int8" else L.veda_attend_fp8
+    reading = O.attend_tiles_int8 if fmt == "int8" else O.attend_tiles_fp8
+    out_p = torch.full((wl.seq_len, wl.heads, wl.dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    out_s = out_p.clone()
+    want = np.zeros((wl.seq_len, wl.heads, wl.dim), np.float64)
+    for box, heads in c.groups:
+        res = c.run_group(box, heads)
+        lay = res["layout"]
+        n = len(heads)
+        q8 = torch.empty(n, lay.n_slots, wl.dim, dtype=code_t, device="cuda")
+        k8 = torch.empty_like(q8)
+        sq = torch.empty(n, lay.n_tiles, dtype=torch.float32, device="cuda")
+        sk = torch.empty_like(sq)
+        row_sq = torch.full((n, wl.seq_len), -1.0, device="cuda")
+        max_sq = torch.full((n,), -1.0, device="cuda")
+        gather(lay, qs, res["heads"], q8, sq, None, row_sq=row_sq)
+        gather(lay, c.dk, res["heads"], k8, sk, None, max_sq=max_sq)
+        row_sq_p, max_sq_p = norms(lay, qs, c.dk, res["heads"], n, wl.seq_len)
+        assert torch.equal(row_sq, row_sq_p) and torch.equal(max_sq, max_sq_p)
+        ws = L.paired_workspace(lay, n)
+        paired(lay, q8, k8, sq, sk, res["v_t"], res["kept_idx"], res["kept_cnt"], out_p, res["heads"], row_sq, max_sq,
+               ws)
+        single(lay, q8, k8, sq, sk, res["v_t"], res["kept_idx"], res["kept_cnt"], out_s, res["heads"])
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        assert q_scale != 1.0 or not redo_flags(lay, n, ws).any()
+        lay_o = O.build_layout(c.spans_oracle(box), wl.seq_len)
+        _, mask = oracle_kept(lay_o, f32(res["scores"]), O.column_blocks(lay_o, wl.generated, wl.reference))
+        qt, kt, vt = (O.gather(x, lay_o, heads) for x in (q, k, v))
+        O.scatter(want, reading(qt, kt, vt, lay_o, lambda hh, i: np.flatnonzero(mask[hh, i])), lay_o, heads)
+    mx, mean = attention_error(f32(out_p), want)
+    assert mx <= ATT_MAX_ABS and mean <= ATT_MEAN_ABS, (mx, mean)
+    assert float((out_p.float() - out_s.float()).abs().max()) <= ATT_MAX_ABS

@@ -207,3 +207,21 @@ def test_published_configurations_take_the_gather_free_path(name):
     for shape, _heads in V.head_groups(wl, lambda _: lps):
         lay = L.veda_plan(spans_ref + [(wl.target[0], wl.target[1], shape)], wl.seq_len, wl.generated, wl.reference)
         assert L.veda_layout_has_box_form(lay), (name, shape)
+
+
+@pytest.mark.parametrize("name", ["tiny", "padded_tiny", "small_d128", "single"])
+@pytest.mark.parametrize("n_heads", [1, 3, 24])
+def test_paired_workspace_size(name, n_heads):
+    # the paired attend's workspace: per head the merged lists of ceil(n_video / 2) pairs (2 max_kept units
+    # each) and their (units, units of A) counts, then a redo flag per (head, tile), the redo list's length
+    # and the redo list, every region 256-byte aligned; host arithmetic only (no device)
+    wl = V.workload(name)
+    lps = O.least_padding_shape(wl.target[1])
+    lay = L.veda_plan([(s, g, None) for s, g in wl.ref_spans] + [(wl.target[0], wl.target[1], lps)], wl.seq_len,
+                      wl.generated, wl.reference)
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    pairs = (lay.n_video + 1) // 2
+    want = (a256(n_heads * pairs * 2 * lay.max_kept * 4) + a256(n_heads * pairs * 8) + 2 * a256(n_heads * lay.n_tiles * 4)
+            + 256)
+    assert L.veda_attend_paired_workspace_bytes(lay, n_heads) == want
+    assert L.veda_attend_paired_workspace_bytes(lay, 0) == 0

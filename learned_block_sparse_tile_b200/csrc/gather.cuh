@@ -40,13 +40,19 @@ struct GatherArgs {
     int64_t seq_len;
 };
 
-template <int D, int kCode = 0>
-__global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
+// CTAs of the pool-only launch (kPoolOnly: no tile copy, veda_pool) resident per SM, which its registers
+// are held to: a pass that only reads keeps more bytes in flight with more CTAs resident.
+constexpr int kPoolCtasPerSm = 4;
+
+template <int D, int kCode = 0, bool kPoolOnly = false>
+__global__ void __launch_bounds__(256, kPoolOnly ? kPoolCtasPerSm : 0) gather_pool_kernel(const GatherArgs a) {
+    static_assert(!(kPoolOnly && kCode != 0), "the 8-bit gathers write codes");
     constexpr int kTpr = D / 8;          // threads per row (8 bf16 = 16 bytes each)
     constexpr int kRpp = 256 / kTpr;     // rows per pass
     constexpr int kPasses = 128 / kRpp;  // passes over the tile
     constexpr int kWarps = 8;
     __shared__ float red[3][kWarps][D];
+    __shared__ unsigned warp_max[kWarps];  // each warp's largest row norm (float bits)
 
     const int tile = blockIdx.x, hh = blockIdx.y;
     const int tid = threadIdx.x, c = tid % kTpr, r0 = tid / kTpr;
@@ -66,7 +72,9 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
         pr[p] = __ldg(a.perm + int64_t(tile) * 128 + r);
         v[p] = pr[p] >= 0 ? __ldg(reinterpret_cast<const uint4*>(src + int64_t(pr[p]) * a.s0)) : make_uint4(0, 0, 0, 0);
     }
-    if (a.row_sq != nullptr || a.max_sq != nullptr) {
+    const bool norms = a.row_sq != nullptr || a.max_sq != nullptr;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (norms) {
         // ||x||^2 per row. Each thread squares its 8 columns of each of its kPasses rows; the kTpr threads
         // of a row then add up with a transposed butterfly: at every step a thread keeps half of its rows
         // and hands the other half to its partner, so the kPasses rows cost kPasses - 1 + log2(kTpr /
@@ -107,30 +115,38 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
         int my_pr = pr[0];
 #pragma unroll
         for (int p = 1; p < kPasses; ++p) my_pr = pm == p ? pr[p] : my_pr;
-        __shared__ unsigned cta_max;
-        if (tid == 0) cta_max = 0u;
-        __syncthreads();
-        if (c < kPasses && my_pr >= 0) {
-            if (a.row_sq != nullptr) a.row_sq[int64_t(hh) * a.seq_len + my_pr] = ss[0];
-            // non-negative floats order as their bit patterns
-            if (a.max_sq != nullptr) atomicMax(&cta_max, __float_as_uint(ss[0]));
-        }
-        if (a.max_sq != nullptr) {
-            __syncthreads();
-            if (tid == 0) atomicMax(a.max_sq + hh, cta_max);
-        }
+        const bool mine = c < kPasses && my_pr >= 0;
+        if (mine && a.row_sq != nullptr) a.row_sq[int64_t(hh) * a.seq_len + my_pr] = ss[0];
+        // non-negative floats order as their bit patterns; the warps' maxima meet after the next barrier
+        const unsigned wm = __reduce_max_sync(0xffffffffu, mine ? __float_as_uint(ss[0]) : 0u);
+        if (lane == 0) warp_max[warp] = wm;
     }
+    // the CTA's largest row norm into max_sq (after a barrier that follows the warp_max writes)
+    auto raise_max = [&]() {
+        if (a.max_sq != nullptr && tid == 0) {
+            unsigned m = 0u;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) m = max(m, warp_max[w]);
+            atomicMax(a.max_sq + hh, m);
+        }
+    };
     const int64_t base = (int64_t(hh) * a.n_slots + int64_t(tile) * 128) * D + c * 8;
     if constexpr (kCode != 0) {
         __shared__ float red8[8];
         quantize_tile<D, kCode>(v, r0, vc, red8, a.codes + base, a.scales + int64_t(hh) * a.n_tiles + tile);
-    } else if (a.x_t != nullptr) {
+    } else if (!kPoolOnly && a.x_t != nullptr) {
         __nv_bfloat16* dst = a.x_t + base;
 #pragma unroll
         for (int p = 0; p < kPasses; ++p) *reinterpret_cast<uint4*>(dst + int64_t(r0 + p * kRpp) * D) = v[p];
     }
 
-    if (a.feats == nullptr || tile >= a.n_video) return;
+    if (a.feats == nullptr || tile >= a.n_video) {
+        if (norms) {
+            __syncthreads();
+            raise_max();
+        }
+        return;
+    }
 
     // column sums in fp32 (packed pairs), maxima and minima on the bf16 pairs themselves (exact either way)
     uint64_t sum2[4];
@@ -175,7 +191,6 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
             mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], off));
         }
     }
-    const int warp = tid >> 5, lane = tid & 31;
     if (lane < kTpr) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -185,6 +200,7 @@ __global__ void __launch_bounds__(256) gather_pool_kernel(const GatherArgs a) {
         }
     }
     __syncthreads();
+    if (norms) raise_max();
     if (tid < D) {
         float s = 0.f, hi = -INFINITY, lo = INFINITY;
 #pragma unroll

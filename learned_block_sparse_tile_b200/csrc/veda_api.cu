@@ -319,9 +319,9 @@ extern "C" int veda_pool(const veda_layout* layout, const void* x, const int64_t
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (int rc = clear_max_sq(max_sq, n_heads, s)) return rc;
     if (dim == 128)
-        gather_pool_kernel<128><<<grid, 256, 0, s>>>(a);
+        gather_pool_kernel<128, 0, true><<<grid, 256, 0, s>>>(a);
     else
-        gather_pool_kernel<64><<<grid, 256, 0, s>>>(a);
+        gather_pool_kernel<64, 0, true><<<grid, 256, 0, s>>>(a);
     return launch_check("gather_pool_kernel");
 }
 

@@ -205,3 +205,41 @@ def _paths_agree(wl, x, paired):
             n = int(c1[h, r])
             assert torch.equal(i1[h, r, :n], i2[h, r, :n])
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("name", ["single", "mixed"])
+def test_pool_equals_gather(name):
+    # veda_pool (the read-only launch of the gather kernel) writes the gather's features, row norms and
+    # per-head maxima bit for bit, on every tile of the full-size layouts, with the heads listed out of order
+    # and one head listed twice; the norms also match float64
+    wl = V.workload(name)
+    x = inputs(wl)
+    lps = O.least_padding_shape(wl.target[1])
+    box, heads = V.head_groups(wl, lambda _: lps)[0]
+    heads = list(heads)[::-1] + [heads[0]]
+    spans_c = [(s, g, None) for s, g in wl.ref_spans] + [(wl.target[0], wl.target[1], box)]
+    lay = L.veda_plan(spans_c, wl.seq_len, wl.generated, wl.reference)
+    n, D = len(heads), wl.dim
+    hd = torch.tensor(heads, dtype=torch.int32, device="cuda")
+    for src in (x["dq"], x["dk"]):
+        f_p = torch.full((n, lay.n_video, 3 * D), -3.0, device="cuda")
+        f_g = torch.full_like(f_p, -5.0)
+        rs_p = torch.full((n, wl.seq_len), -1.0, device="cuda")
+        rs_g = torch.full_like(rs_p, -2.0)
+        mx_p = torch.full((n,), -1.0, device="cuda")
+        mx_g = torch.full_like(mx_p, -2.0)
+        x_t = torch.empty(n, lay.n_slots, D, dtype=torch.bfloat16, device="cuda")
+        L.veda_pool(lay, src, hd, f_p, row_sq=rs_p, max_sq=mx_p)
+        L.veda_gather(lay, src, hd, x_t, f_g, row_sq=rs_g, max_sq=mx_g)
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        assert torch.equal(f_p, f_g)
+        assert torch.equal(rs_p, rs_g)
+        assert torch.equal(mx_p, mx_g)
+        # without norms (video tiles only) the features are the same
+        f_p2 = torch.full_like(f_p, -7.0)
+        L.veda_pool(lay, src, hd, f_p2)
+        assert L.veda_sync_status() == L.VEDA_OK, L.veda_last_error()
+        assert torch.equal(f_p2, f_g)
+        sq = torch.stack([(src[:, h, :].double() ** 2).sum(-1) for h in heads])  # [n, S], float64
+        assert torch.allclose(rs_p.double(), sq, rtol=1e-5, atol=0)
+        assert torch.allclose(mx_p.double(), sq.max(1).values, rtol=1e-5, atol=0)

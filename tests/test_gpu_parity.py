@@ -548,6 +548,7 @@ def test_logit_bound(name, q_scale):
             assert np.allclose(f32(got), want_q, rtol=1e-5, atol=0)
         for got in (max_sq, max_sq_g):
             assert np.allclose(f32(got), want_k, rtol=1e-5, atol=0)
+        assert torch.equal(row_sq, row_sq_g) and torch.equal(max_sq, max_sq_g)
         L.veda_attend_direct(lay, qs, c.dk, c.dv, res["kept_idx"], res["kept_cnt"], out_d, res["heads"],
                              q_row_sq=row_sq, k_max_sq=max_sq)
         L.veda_attend(lay, q_t, k_t, res["v_t"], res["kept_idx"], res["kept_cnt"], out_t, res["heads"],

@@ -216,11 +216,14 @@ int veda_pool(const veda_layout* layout, const void* x, const int64_t x_strides[
               int32_t dim, const int32_t* heads, int32_t n_heads, float* feats, float* row_sq, float* max_sq,
               void* stream);
 
-/* Workspace bytes veda_score needs (projected features of Q and K): 2 * n_heads * n_video * D * 4. */
+/* Workspace bytes veda_score needs (projected features of Q and K, and both projections transposed):
+ * n_heads * (2 * n_video * D + 6 * D * D) * 4. */
 size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim);
 
 /* Tile-pair logits (veda_core.py, "predictor", logits): per head, q_hat = fq @ Pq + fq[:, :D],
- * k_hat = fk @ Pk + fk[:, :D], scores = q_hat @ k_hat^T / sqrt(D), all fp32.
+ * k_hat = fk @ Pk + fk[:, :D], scores = q_hat @ k_hat^T / sqrt(D), all fp32 (on the tensor cores as split tf32:
+ * each operand as a tf32 high part and its fp32 remainder, three tf32 products per product, which keeps the
+ * error at the level of fp32 rounding).
  *  feats_q/k  device fp32 [n_heads, n_video, 3D] (from veda_gather).
  *  proj_q/k   device fp32 [n_heads, 3D, D]: the group's heads' projections, in the group's head order.
  *  workspace  device, at least veda_score_workspace_bytes(), 16-byte aligned.
@@ -233,7 +236,8 @@ int veda_score(const veda_layout* layout, const float* feats_q, const float* fea
  * need the scores: plugins whose device memory belongs to a pool the host application owns and budgets,
  * and real-time loops where an allocation, which can block on or synchronise with the device, is not
  * allowed. The pages have no counterpart: this is a service of this library.
- * Same inputs, outputs and arithmetic as veda_score; the projected features live in one 4 MiB array of
+ * Same inputs, outputs and arithmetic as veda_score; the projected features (and the transposed
+ * projections) live in one 4 MiB array of
  * this library's device memory (1,048,576 floats, held by every GPU that loads the library until exit)
  * and heads are processed in chunks that fit it. Nothing is allocated and nothing needs to start at zero.
  * The first call on a device looks up the array's device address and keeps it for the process's life
@@ -241,7 +245,7 @@ int veda_score(const veda_layout* layout, const float* feats_q, const float* fea
  * call this entry point again in that process).
  * All calls on a device share the array: calls whose kernels overlap on the GPU race and must be
  * serialised. Errors: VEDA_ERR_UNSUPPORTED when one head needs more than the array holds
- * (2 * n_video * D > 1,048,576, i.e. n_video > 4096 at D = 128); otherwise as veda_score. */
+ * (2 * n_video * D + 6 * D * D > 1,048,576, i.e. n_video > 3712 at D = 128); otherwise as veda_score. */
 int veda_score_noalloc(const veda_layout* layout, const float* feats_q, const float* feats_k, int32_t n_heads,
                        int32_t dim, const float* proj_q, const float* proj_k, float* scores, void* stream);
 

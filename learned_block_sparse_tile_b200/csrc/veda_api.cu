@@ -38,6 +38,7 @@ struct DeviceState {
     int* err = nullptr;  // device address of g_err
     bool attend_attr[8] = {};  // (head_dim 128) + 2 * Q/K format; 6 + (head_dim 128) for the gather-free variant
     bool pair_attr[12] = {};   // paired kernel: (head_dim 128) + 2 * gather-free + 4 * Q/K format
+    bool score_attr = false;   // the score GEMM's shared-memory size is set
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -394,8 +395,92 @@ extern "C" int veda_gather_int8(const veda_layout* layout, const void* x, const 
 
 extern "C" size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, int32_t dim) {
     if (!layout || n_heads <= 0 || dim <= 0) return 0;
-    return size_t(2) * size_t(n_heads) * size_t(layout->desc.n_video) * size_t(dim) * sizeof(float);
+    return size_t(n_heads) * size_t(score_scratch_per_head(layout->desc.n_video, dim)) * sizeof(float);
 }
+
+namespace veda {
+
+// 3D fp32 map over [batch][rows][K] (K innermost): boxes of 32 K-columns (128 bytes) x 128 rows with the
+// 128-byte swizzle of the tf32 MMA operands; rows past `rows` read as zeros.
+int make_f32_map(CUtensorMap* m, const float* base, int64_t K, int64_t rows, int64_t batch) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t gdim[3] = {cuuint64_t(K), cuuint64_t(rows), cuuint64_t(batch)};
+    cuuint64_t gstride[2] = {cuuint64_t(K) * 4, cuuint64_t(rows) * cuuint64_t(K) * 4};
+    cuuint32_t box[3] = {cuuint32_t(tf32x3::kBK), cuuint32_t(tf32x3::kBM), 1};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled (fp32 operand) failed (" + std::to_string(int(r)) + ")");
+    return VEDA_OK;
+}
+
+int launch_score_gemms(const float* feats_q, const float* feats_k, const float* proj_q, const float* proj_k, float* qh,
+                       float* kh, float* pt_q, float* pt_k, float* scores, int nv, int dim, int n_heads,
+                       cudaStream_t s) {
+    DeviceState* ds;
+    if (int rc = device_state(&ds)) return rc;
+    if (!ds->score_attr) {
+        cudaError_t e = cudaFuncSetAttribute(tf32x3::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(tf32x3::kSmem));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(score gemm_kernel)");
+        ds->score_attr = true;
+    }
+    if (nv <= 0) return VEDA_OK;
+    // (P + E)^T: both operands of the projection K-major, the residual feats[:, :D] folded in
+    tf32x3::transpose_kernel<<<dim3(unsigned(dim / 32), unsigned(3 * dim / 32), unsigned(2 * n_heads)), 256, 0, s>>>(
+        proj_q, proj_k, pt_q, pt_k, n_heads, 3 * dim, dim);
+    if (int rc = launch_check("score transpose_kernel")) return rc;
+
+    // q_hat = fq (P_q + E) = fq P_q + fq[:, :D] and k_hat likewise, in one launch (two operand sets)
+    tf32x3::Maps pm;
+    if (int rc = make_f32_map(&pm.a[0], feats_q, 3 * dim, nv, n_heads)) return rc;
+    if (int rc = make_f32_map(&pm.b[0], pt_q, 3 * dim, dim, n_heads)) return rc;
+    if (int rc = make_f32_map(&pm.a[1], feats_k, 3 * dim, nv, n_heads)) return rc;
+    if (int rc = make_f32_map(&pm.b[1], pt_k, 3 * dim, dim, n_heads)) return rc;
+    tf32x3::Args pa{};
+    pa.n_sets = 2;
+    pa.nb = n_heads;
+    pa.M = nv;
+    pa.N = dim;
+    pa.K = 3 * dim;
+    pa.tiles_m = (nv + tf32x3::kBM - 1) / tf32x3::kBM;
+    pa.tiles_n = 1;
+    pa.n_tiles = 2 * n_heads * pa.tiles_m;
+    pa.C[0] = qh;
+    pa.C[1] = kh;
+    pa.scale = 1.f;
+    pa.timeout_ns = g_timeout_ns.load();
+    pa.err = ds->err;
+    tf32x3::gemm_kernel<<<unsigned(std::min(pa.n_tiles, ds->sms)), tf32x3::kThreads, tf32x3::kSmem, s>>>(pm, pa);
+    if (int rc = launch_check("score gemm_kernel (projections)")) return rc;
+
+    // scores = q_hat k_hat^T / sqrt(D), as a product with 1 / sqrt(D) rounded to fp32
+    tf32x3::Maps lm;
+    if (int rc = make_f32_map(&lm.a[0], qh, dim, nv, n_heads)) return rc;
+    if (int rc = make_f32_map(&lm.b[0], kh, dim, nv, n_heads)) return rc;
+    lm.a[1] = lm.a[0];
+    lm.b[1] = lm.b[0];
+    tf32x3::Args la{};
+    la.n_sets = 1;
+    la.nb = n_heads;
+    la.M = nv;
+    la.N = nv;
+    la.K = dim;
+    la.tiles_m = (nv + tf32x3::kBM - 1) / tf32x3::kBM;
+    la.tiles_n = (nv + tf32x3::kBN - 1) / tf32x3::kBN;
+    la.n_tiles = n_heads * la.tiles_m * la.tiles_n;
+    la.C[0] = la.C[1] = scores;
+    la.scale = float(1.0 / std::sqrt(double(dim)));
+    la.timeout_ns = pa.timeout_ns;
+    la.err = ds->err;
+    tf32x3::gemm_kernel<<<unsigned(std::min(la.n_tiles, ds->sms)), tf32x3::kThreads, tf32x3::kSmem, s>>>(lm, la);
+    return launch_check("score gemm_kernel (logits)");
+}
+
+}  // namespace veda
 
 extern "C" int veda_score(const veda_layout* layout, const float* feats_q, const float* feats_k, int32_t n_heads,
                           int32_t dim, const float* proj_q, const float* proj_k, void* workspace,
@@ -415,9 +500,10 @@ extern "C" int veda_score(const veda_layout* layout, const float* feats_q, const
     const int nv = layout->desc.n_video;
     float* qh = static_cast<float*>(workspace);
     float* kh = qh + int64_t(n_heads) * nv * dim;
+    float* pt_q = kh + int64_t(n_heads) * nv * dim;
+    float* pt_k = pt_q + int64_t(n_heads) * 3 * dim * dim;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    launch_score_gemms(feats_q, feats_k, proj_q, proj_k, qh, kh, scores, nv, dim, n_heads, s);
-    return launch_check("gemm_f32_kernel");
+    return launch_score_gemms(feats_q, feats_k, proj_q, proj_k, qh, kh, pt_q, pt_k, scores, nv, dim, n_heads, s);
 }
 
 template <int kPer>

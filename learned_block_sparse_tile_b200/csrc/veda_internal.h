@@ -1,6 +1,8 @@
 // Internal declarations of libveda (not part of the C ABI).
 #pragma once
 
+#include <cuda_runtime.h>
+
 #include <cstdint>
 #include <mutex>
 #include <string>
@@ -36,6 +38,17 @@ struct DeviceCopy {
 // Records `msg` as the calling thread's last error and returns `code`.
 int fail(int code, const std::string& msg);
 void clear_error();
+
+// Floats of scratch the predictor's products need per head: the projected q and k features (2 n_video D)
+// and the two projections transposed (2 x 3D x D).
+inline int64_t score_scratch_per_head(int64_t n_video, int64_t dim) { return 2 * n_video * dim + 6 * dim * dim; }
+
+// Enqueues the predictor's products for n_heads heads on `s` (veda_score's arithmetic): P^T into pt_q /
+// pt_k ([n_heads][D][3D]), q_hat / k_hat into qh / kh ([n_heads][n_video][D]), then the scores
+// ([n_heads][n_video][n_video]). All pointers 16-byte aligned device memory. Returns a VEDA_* status.
+int launch_score_gemms(const float* feats_q, const float* feats_k, const float* proj_q, const float* proj_k, float* qh,
+                       float* kh, float* pt_q, float* pt_k, float* scores, int nv, int dim, int n_heads,
+                       cudaStream_t s);
 
 }  // namespace veda
 

@@ -4,8 +4,8 @@
 // whose device memory is owned and budgeted by the host application's own pool (a plugin may not grow it),
 // and real-time loops where an allocation is not allowed because it can block on, or synchronise with,
 // the device. veda_score asks its caller for a workspace; this entry point instead keeps that scratch (the
-// projected query and key features) in one fixed array in this library's device memory, and the caller
-// passes only its inputs and outputs.
+// projected query and key features and the transposed projections) in one fixed array in this library's
+// device memory, and the caller passes only its inputs and outputs.
 //
 // The scratch is a file-scope __device__ array of kScratchFloats floats (4 MiB). Every GPU that loads
 // the library holds it until the process exits. All calls on a device share it; it keeps whatever the
@@ -25,7 +25,6 @@
 #include <string>
 
 #include "veda_internal.h"
-#include "score.cuh"
 
 namespace {
 
@@ -54,10 +53,11 @@ extern "C" int veda_score_noalloc(const veda_layout* layout, const float* feats_
     if (!aligned16(feats_q) || !aligned16(feats_k) || !aligned16(proj_q) || !aligned16(proj_k) || !aligned16(scores))
         return veda::fail(VEDA_ERR_INVALID, "veda_score_noalloc: buffers need 16-byte alignment");
     const int64_t nv = layout->desc.n_video;
-    const size_t per_head = size_t(2) * size_t(nv) * size_t(dim);  // projected q and k of one head
+    const size_t per_head = size_t(veda::score_scratch_per_head(nv, dim));
     if (per_head > kScratchFloats)
         return veda::fail(VEDA_ERR_UNSUPPORTED,
-                          "veda_score_noalloc: one head needs 2 * n_video * head_dim = " + std::to_string(per_head) +
+                          "veda_score_noalloc: one head needs 2 * n_video * head_dim + 6 * head_dim^2 = " +
+                              std::to_string(per_head) +
                               " floats of scratch but the static scratch holds " + std::to_string(kScratchFloats) +
                               " (4 MiB); use veda_score with a caller-provided workspace");
     if (int rc = veda_device_check()) return rc;
@@ -88,13 +88,13 @@ extern "C" int veda_score_noalloc(const veda_layout* layout, const float* feats_
     for (int h0 = 0; h0 < n_heads; h0 += chunk) {
         const int hc = std::min(chunk, n_heads - h0);
         float* qh = base;
-        float* kh = base + int64_t(hc) * nv * dim;
-        veda::launch_score_gemms(feats_q + int64_t(h0) * nv * 3 * dim, feats_k + int64_t(h0) * nv * 3 * dim,
-                                 proj_q + int64_t(h0) * 3 * dim * dim, proj_k + int64_t(h0) * 3 * dim * dim, qh, kh,
-                                 scores + int64_t(h0) * nv * nv, int(nv), dim, hc, s);
+        float* kh = qh + int64_t(hc) * nv * dim;
+        float* pt_q = kh + int64_t(hc) * nv * dim;
+        float* pt_k = pt_q + int64_t(hc) * 3 * dim * dim;
+        if (int rc = veda::launch_score_gemms(feats_q + int64_t(h0) * nv * 3 * dim, feats_k + int64_t(h0) * nv * 3 * dim,
+                                              proj_q + int64_t(h0) * 3 * dim * dim, proj_k + int64_t(h0) * 3 * dim * dim,
+                                              qh, kh, pt_q, pt_k, scores + int64_t(h0) * nv * nv, int(nv), dim, hc, s))
+            return rc;
     }
-    e = cudaGetLastError();
-    if (e != cudaSuccess)
-        return veda::fail(VEDA_ERR_CUDA, std::string("veda_score_noalloc launch: ") + cudaGetErrorString(e));
     return VEDA_OK;
 }

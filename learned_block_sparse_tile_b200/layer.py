@@ -37,8 +37,9 @@ class VedaLayer:
                  keeps the single-tile attend
     """
 
-    LAUNCHES_PER_GROUP = 7  # tile-order path: gather q, gather k, 2 score GEMMs, select, gather v, attend
-    LAUNCHES_PER_GROUP_DIRECT = 6  # gather-free path: pool q, pool k, 2 score GEMMs, select, attend
+    # tile-order path: gather q, gather k, the projections' transpose, 2 score GEMMs, select, gather v, attend
+    LAUNCHES_PER_GROUP = 8
+    LAUNCHES_PER_GROUP_DIRECT = 7  # gather-free path: pool q, pool k, transpose, 2 score GEMMs, select, attend
     EXTRA_LAUNCHES_PAIRED = 2  # the paired attend adds the list merge and the (usually empty) redo pass
 
     def __init__(self, seq_len, ref_spans, target, head_shapes, budgets, heads, dim, device="cuda", fp8_qk=False,

@@ -225,3 +225,16 @@ def test_paired_workspace_size(name, n_heads):
             + 256)
     assert L.veda_attend_paired_workspace_bytes(lay, n_heads) == want
     assert L.veda_attend_paired_workspace_bytes(lay, 0) == 0
+
+
+@pytest.mark.parametrize("name,n_heads,dim", [("small_d128", 3, 128), ("single", 24, 128), ("small_d128", 2, 64)])
+def test_score_workspace_size(name, n_heads, dim):
+    # veda_score's workspace: per head the projected q and k features (2 n_video D floats) and both
+    # projections transposed with the residual's identity block ((P + E)^T, 2 x D x 3D floats); host only
+    wl = V.workload(name)
+    lps = O.least_padding_shape(wl.target[1])
+    lay = L.veda_plan([(s, g, None) for s, g in wl.ref_spans] + [(wl.target[0], wl.target[1], lps)], wl.seq_len,
+                      wl.generated, wl.reference)
+    want = n_heads * (2 * lay.n_video * dim + 2 * dim * 3 * dim) * 4
+    assert L.veda_score_workspace_bytes(lay, n_heads, dim) == want
+    assert L.veda_score_workspace_bytes(lay, 0, dim) == 0

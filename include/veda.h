@@ -226,8 +226,12 @@ size_t veda_score_workspace_bytes(const veda_layout* layout, int32_t n_heads, in
  * error at the level of fp32 rounding).
  *  feats_q/k  device fp32 [n_heads, n_video, 3D] (from veda_gather).
  *  proj_q/k   device fp32 [n_heads, 3D, D]: the group's heads' projections, in the group's head order.
- *  workspace  device, at least veda_score_workspace_bytes(), 16-byte aligned.
- *  scores     device fp32 [n_heads, n_video, n_video] out. */
+ *  workspace  device, at least veda_score_workspace_bytes(), 16-byte aligned; caller-owned scratch (the
+ *             projected features and the transposed projections), overwritten by every call.
+ *  scores     device fp32 [n_heads, n_video, n_video] out.
+ * Errors: VEDA_ERR_INVALID for NULL or unaligned buffers, a workspace below the size, D other than 64 or
+ * 128 or n_heads <= 0; VEDA_ERR_CUDA when a launch or a tensor-map encoding fails. The kernels' waits are
+ * bounded: one that expires stops the kernel early and veda_sync_status reports VEDA_ERR_TIMEOUT. */
 int veda_score(const veda_layout* layout, const float* feats_q, const float* feats_k, int32_t n_heads,
                int32_t dim, const float* proj_q, const float* proj_k, void* workspace,
                size_t workspace_bytes, float* scores, void* stream);

@@ -5,8 +5,9 @@
 // Split tf32. A tf32 operand keeps 10 explicit mantissa bits, too few for fp32 scores on its own, so every
 // operand x is split into hi = x rounded to tf32 and lo = x - hi (exact in fp32, |lo| <= 2^-11 |x|), and
 // a b is taken as hi_a hi_b + hi_a lo_b + lo_a hi_b: three kind::tf32 products into one fp32 accumulator.
-// What is left out, lo_a lo_b and the bits of the lo parts below tf32, is under 2^-21 |a b| per product:
-// the order of the rounding of an fp32 dot product itself.
+// What is left out, lo_a lo_b (under 2^-22 |a b|) and the bits of the lo parts below tf32 (each under
+// 2^-21 |a b| even if the MMA truncates them), is under 1.25 x 2^-20 |a b| per product: the order of the
+// rounding of an fp32 dot product itself.
 //
 // Both products are C[batch] = scale A[batch] B[batch]^T with A [M][K] and B [N][K] K-major fp32. The
 // projection's B is (P + E)^T, written first by transpose_kernel, where E is the identity in P's first D
